@@ -1,0 +1,250 @@
+"""B200 (sm_100a) denoising step of block discrete-diffusion text generation.
+
+A thin ctypes binding of ``libdg.so`` (C ABI in ``include/dg.h``): argument
+marshalling only.  Every step of the path runs in the library's CUDA
+kernels; PyTorch supplies device memory and streams.  There is no CPU
+fallback: if the library is missing or no sm_100 device is present, calls
+raise ``DGError``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import numpy as np
+
+__all__ = ["DGError", "Params", "lib", "workspace_size", "Workspace", "denoise_step",
+           "debug_logits", "device_status", "denoise_loop", "debug_gumbel",
+           "selftest_bounded_wait", "STATUS", "E_BF16", "E_FP8_E4M3"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdg.so")
+
+E_BF16 = 0
+E_FP8_E4M3 = 1
+
+STATUS = {0: "DG_OK", 1: "DG_ERR_INVALID_ARG", 2: "DG_ERR_UNSUPPORTED_SHAPE", 3: "DG_ERR_WORKSPACE",
+          4: "DG_ERR_RANGE", 5: "DG_ERR_CUDA", 6: "DG_ERR_TIMEOUT", 7: "DG_ERR_CALLBACK",
+          8: "DG_ERR_NO_DEVICE"}
+
+
+class DGError(RuntimeError):
+    def __init__(self, code: int, where: str = ""):
+        self.code = int(code)
+        super().__init__(f"{where}: {STATUS.get(self.code, self.code)}")
+
+
+class _Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("L", ctypes.c_int32), ("d", ctypes.c_int32),
+                ("V", ctypes.c_int32), ("e_dtype", ctypes.c_int32)]
+
+
+class _Params(ctypes.Structure):
+    _fields_ = [("tau0", ctypes.c_double), ("tau1", ctypes.c_double), ("max_steps", ctypes.c_int32),
+                ("entropy_bound", ctypes.c_double), ("stop_entropy", ctypes.c_double),
+                ("seed", ctypes.c_uint64)]
+
+
+_HIDDEN_FN = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
+                              ctypes.c_void_p, ctypes.c_void_p)
+
+
+@dataclass
+class Params:
+    """Sampler parameters (defaults: the serving configuration of the docs)."""
+    tau0: float = 0.8
+    tau1: float = 0.4
+    max_steps: int = 48
+    entropy_bound: float = 0.1
+    stop_entropy: float = 0.005
+    seed: int = 1234
+
+    def c(self) -> _Params:
+        return _Params(self.tau0, self.tau1, self.max_steps, self.entropy_bound,
+                       self.stop_entropy, int(self.seed) & 0xFFFFFFFFFFFFFFFF)
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libdg.so (built in-tree by ``block_canvas_denoising_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise DGError(5, f"libdg.so not built at {LIB_PATH}")
+        L = ctypes.CDLL(LIB_PATH)
+        P = ctypes.c_void_p
+        L.dg_default_params.restype = _Params
+        L.dg_error_string.restype = ctypes.c_char_p
+        L.dg_error_string.argtypes = [ctypes.c_int]
+        L.dg_workspace_size.restype = ctypes.c_size_t
+        L.dg_workspace_size.argtypes = [ctypes.POINTER(_Shape)]
+        L.dg_workspace_init.argtypes = [P, ctypes.c_size_t, P]
+        step_args = [ctypes.POINTER(_Shape), ctypes.POINTER(_Params), P, P, P, P, P, P,
+                     P, P, P, P, P, P, P]
+        L.dg_denoise_step.argtypes = step_args + [P, ctypes.c_size_t, P]
+        L.dg_debug_logits.argtypes = step_args + [P, P, ctypes.c_size_t, P]
+        L.dg_device_status.argtypes = [P, ctypes.c_size_t, P]
+        L.dg_denoise_loop.argtypes = [ctypes.POINTER(_Shape), ctypes.POINTER(_Params), P, P,
+                                      _HIDDEN_FN, P, ctypes.c_int32, P, P, P, P, P,
+                                      P, P, P, P, P, P, ctypes.c_size_t, P]
+        L.dg_selftest_bounded_wait.argtypes = [ctypes.c_uint64, P, ctypes.c_size_t, P]
+        L.dg_debug_gumbel.argtypes = [P, ctypes.c_int32, P, P, P]
+        for name in ("dg_workspace_init", "dg_denoise_step", "dg_debug_logits", "dg_device_status",
+                     "dg_denoise_loop", "dg_selftest_bounded_wait", "dg_debug_gumbel"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(code: int, where: str) -> None:
+    if code != 0:
+        raise DGError(code, where)
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _host(a, dtype) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=dtype))
+
+
+def _shape(B: int, d: int, V: int, e_dtype: int = E_BF16, L: int = 256) -> _Shape:
+    return _Shape(B, L, d, V, e_dtype)
+
+
+def workspace_size(B: int, d: int, V: int, e_dtype: int = E_BF16, L: int = 256) -> int:
+    """Bytes of workspace one step needs on the current device (0 if invalid)."""
+    return int(lib().dg_workspace_size(ctypes.byref(_shape(B, d, V, e_dtype, L))))
+
+
+class Workspace:
+    """Device scratch for steps of one shape (a zeroed torch uint8 buffer)."""
+
+    def __init__(self, B: int, d: int, V: int, e_dtype: int = E_BF16, device=None, stream=None):
+        import torch
+        n = workspace_size(B, d, V, e_dtype)
+        if n == 0:
+            raise DGError(2, "workspace_size")
+        self.nbytes = n
+        self.buf = torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+        _check(lib().dg_workspace_init(_ptr(self.buf), ctypes.c_size_t(n), _stream(stream)),
+               "dg_workspace_init")
+
+
+def _step_call(fn_name, h, E, step_idx, has_prev, canvas, prev_argmax, accept, entropy, sampled,
+               argmax, stop, ws: Workspace, params: Params, e_scale=None, active=None, logits=None,
+               stream=None):
+    B = int(len(step_idx))
+    R, d = h.shape
+    V = E.shape[0]
+    e_dtype = E_BF16 if e_scale is None else E_FP8_E4M3
+    shp = _shape(B, d, V, e_dtype, L=R // max(B, 1))
+    prm = params.c()
+    ks = _host(step_idx, np.int32)
+    hp = _host(has_prev, np.uint8)
+    act = None if active is None else _host(active, np.uint8)
+    args = [ctypes.byref(shp), ctypes.byref(prm), _ptr(h), _ptr(E), _ptr(e_scale),
+            ks.ctypes.data_as(ctypes.c_void_p), hp.ctypes.data_as(ctypes.c_void_p),
+            None if act is None else act.ctypes.data_as(ctypes.c_void_p),
+            _ptr(canvas), _ptr(prev_argmax), _ptr(accept), _ptr(entropy), _ptr(sampled),
+            _ptr(argmax), _ptr(stop)]
+    if fn_name == "dg_debug_logits":
+        args.append(_ptr(logits))
+    args += [_ptr(ws.buf), ctypes.c_size_t(ws.nbytes), _stream(stream)]
+    _check(getattr(lib(), fn_name)(*args), fn_name)
+
+
+def denoise_step(h, E, step_idx, has_prev, canvas, prev_argmax, accept, entropy, sampled, argmax,
+                 stop, ws: Workspace, params: Params = Params(), e_scale=None, active=None,
+                 stream=None) -> None:
+    """Enqueue one step (see ``dg_denoise_step`` in include/dg.h).
+
+    Tensors are CUDA tensors: h bf16 [B*256, d], E bf16 [V, d] (or uint8
+    E4M3 codes with ``e_scale`` float [V]), canvas / prev_argmax / sampled /
+    argmax int32 [B*256], accept uint8 [B*256], entropy float32 [B*256],
+    stop int32 [B].  ``step_idx``, ``has_prev`` and ``active`` are host
+    sequences of length B."""
+    _step_call("dg_denoise_step", h, E, step_idx, has_prev, canvas, prev_argmax, accept, entropy,
+               sampled, argmax, stop, ws, params, e_scale, active, None, stream)
+
+
+def debug_logits(h, E, step_idx, has_prev, canvas, prev_argmax, accept, entropy, sampled, argmax,
+                 stop, logits, ws: Workspace, params: Params = Params(), e_scale=None, active=None,
+                 stream=None) -> None:
+    """The same step, also writing the float32 logits [B*256, V] it consumed."""
+    _step_call("dg_debug_logits", h, E, step_idx, has_prev, canvas, prev_argmax, accept, entropy,
+               sampled, argmax, stop, ws, params, e_scale, active, logits, stream)
+
+
+def device_status(ws: Workspace, stream=None) -> int:
+    """Synchronise and read/clear the device fault latch (0 = clean)."""
+    return int(lib().dg_device_status(_ptr(ws.buf), ctypes.c_size_t(ws.nbytes), _stream(stream)))
+
+
+def denoise_loop(E, hidden_fn, h_buf, canvas, prev_argmax, has_prev, accept, entropy, sampled,
+                 argmax, stop, ws: Workspace, params: Params = Params(), k_start: int = 0,
+                 e_scale=None, stream=None):
+    """Run the adaptive loop (``dg_denoise_loop``).
+
+    ``hidden_fn(k, canvas_tensor, h_buf)`` must fill ``h_buf`` for step k on
+    the current stream and return None.  ``has_prev`` is a host uint8 numpy
+    array [B] updated in place.  Returns the host int32 array of steps taken.
+    """
+    B = int(len(has_prev))
+    R, d = h_buf.shape
+    V = E.shape[0]
+    e_dtype = E_BF16 if e_scale is None else E_FP8_E4M3
+    shp = _shape(B, d, V, e_dtype, L=R // B)
+    prm = params.c()
+    steps = np.zeros(B, np.int32)
+    assert isinstance(has_prev, np.ndarray) and has_prev.dtype == np.uint8
+    errors = []
+
+    def cb(k, canvas_ptr, h_ptr, user, stream_ptr):
+        try:
+            hidden_fn(int(k), canvas, h_buf)
+            return 0
+        except Exception as exc:  # reported as DG_ERR_CALLBACK
+            errors.append(exc)
+            return 1
+
+    cfn = _HIDDEN_FN(cb)
+    code = lib().dg_denoise_loop(
+        ctypes.byref(shp), ctypes.byref(prm), _ptr(E), _ptr(e_scale), cfn, None,
+        ctypes.c_int32(k_start), _ptr(h_buf), _ptr(canvas), _ptr(prev_argmax),
+        has_prev.ctypes.data_as(ctypes.c_void_p), steps.ctypes.data_as(ctypes.c_void_p),
+        _ptr(accept), _ptr(entropy), _ptr(sampled), _ptr(argmax), _ptr(stop), _ptr(ws.buf),
+        ctypes.c_size_t(ws.nbytes), _stream(stream))
+    if code != 0:
+        err = DGError(code, "dg_denoise_loop")
+        if errors:
+            raise err from errors[0]
+        raise err
+    return steps
+
+
+def debug_gumbel(words, stream=None):
+    """Device g32 and approximate lg2(E) for uint32 words (torch int32 CUDA tensor)."""
+    import torch
+    n = int(words.numel())
+    g = torch.empty(n, dtype=torch.float32, device=words.device)
+    a = torch.empty(n, dtype=torch.float32, device=words.device)
+    _check(lib().dg_debug_gumbel(_ptr(words), ctypes.c_int32(n), _ptr(g), _ptr(a), _stream(stream)),
+           "dg_debug_gumbel")
+    return g, a
+
+
+def selftest_bounded_wait(limit_ns: int, ws: Workspace, stream=None) -> int:
+    """Run the bounded-wait self test; returns the status code (6 = timed out as designed)."""
+    return int(lib().dg_selftest_bounded_wait(ctypes.c_uint64(limit_ns), _ptr(ws.buf),
+                                              ctypes.c_size_t(ws.nbytes), _stream(stream)))

@@ -1,0 +1,360 @@
+// dg_api.cu -- host side of the C ABI declared in include/dg.h: argument
+// checks, the temperature schedule, TMA descriptors, kernel launches and the
+// adaptive loop.
+#include <cudaTypedefs.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "dg_device.cuh"
+#include "dg_internal.h"
+
+namespace dg {
+
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Current device's SM count, or -1 when it is not an sm_100 part.
+int device_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  int major = 0, sms = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return -1;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  if (major != 10) return -1;
+  return sms;
+}
+
+dg_status check_shape(const dg_shape* s) {
+  if (s == nullptr) return DG_ERR_INVALID_ARG;
+  if (s->B < 1 || s->B > DG_MAX_B || s->L != 256 || s->d < kBlockK || s->d % kBlockK != 0 ||
+      s->V < kBlockN || s->V % kBlockN != 0)
+    return DG_ERR_UNSUPPORTED_SHAPE;
+  if (s->e_dtype != DG_E_BF16) return DG_ERR_UNSUPPORTED_SHAPE;
+  return DG_OK;
+}
+
+bool finite_pos(double x) { return x > 0.0 && x < 1e300; }
+
+dg_status check_params(const dg_params* p) {
+  if (p == nullptr) return DG_ERR_INVALID_ARG;
+  if (p->max_steps < 1 || !finite_pos(p->tau0) || !finite_pos(p->tau1)) return DG_ERR_INVALID_ARG;
+  if (!(p->entropy_bound >= 0.0 && p->entropy_bound < 1e300)) return DG_ERR_INVALID_ARG;
+  if (!(p->stop_entropy >= 0.0 && p->stop_entropy < 1e300)) return DG_ERR_INVALID_ARG;
+  return DG_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Temperature of step k ([Docs] "DiffusionGemma", Recommended serving
+// configuration, temperature schedule: linear from tau0 to tau1 over the N
+// steps), in float64, and its float32 reciprocal.
+float inv_tau_of(const dg_params& p, int k) {
+  double tau;
+  if (p.max_steps == 1) {
+    tau = p.tau0;
+  } else {
+    const double span = (p.tau0 - p.tau1) * static_cast<double>(k);
+    tau = p.tau0 - span / static_cast<double>(p.max_steps - 1);
+  }
+  return static_cast<float>(1.0 / tau);
+}
+
+bool encode_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
+                    uint32_t box_inner, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+struct StepArgs {
+  const dg_shape* shape;
+  const dg_params* params;
+  const void* h;
+  const void* E;
+  const float* e_scale;
+  const int32_t* step_idx;
+  const uint8_t* has_prev;
+  const uint8_t* active;
+  int32_t* canvas;
+  int32_t* prev_argmax;
+  uint8_t* accept;
+  float* entropy;
+  int32_t* sampled;
+  int32_t* argmax;
+  int32_t* stop;
+  float* logits;
+  void* workspace;
+  size_t ws_bytes;
+  cudaStream_t stream;
+};
+
+dg_status run_step(const StepArgs& a) {
+  dg_status st = check_shape(a.shape);
+  if (st != DG_OK) return st;
+  if ((st = check_params(a.params)) != DG_OK) return st;
+  const dg_shape& s = *a.shape;
+  const dg_params& pr = *a.params;
+  if (!a.h || !a.E || !a.step_idx || !a.has_prev || !a.canvas || !a.prev_argmax || !a.accept ||
+      !a.entropy || !a.sampled || !a.argmax || !a.stop || !a.workspace)
+    return DG_ERR_INVALID_ARG;
+  if (!aligned16(a.h) || !aligned16(a.E) || !aligned16(a.workspace)) return DG_ERR_INVALID_ARG;
+  if (a.logits != nullptr && !aligned16(a.logits)) return DG_ERR_INVALID_ARG;
+  for (int b = 0; b < s.B; ++b)
+    if (a.step_idx[b] < 0 || a.step_idx[b] >= pr.max_steps) return DG_ERR_RANGE;
+  const int sms = device_sms();
+  if (sms <= 0) return DG_ERR_NO_DEVICE;
+  const WsLayout ws = ws_layout(s, sms);
+  if (a.ws_bytes < ws.total) return DG_ERR_WORKSPACE;
+
+  const int R = s.B * s.L;
+  uint8_t* wsb = static_cast<uint8_t*>(a.workspace);
+
+  CanvasParam cps[DG_MAX_B];
+  memset(cps, 0, sizeof(cps));
+  for (int b = 0; b < s.B; ++b) {
+    cps[b].k = a.step_idx[b];
+    cps[b].inv_tau = inv_tau_of(pr, a.step_idx[b]);
+    cps[b].has_prev = a.has_prev[b] ? 1 : 0;
+    cps[b].active = (a.active == nullptr || a.active[b]) ? 1 : 0;
+  }
+
+  CUtensorMap tmA, tmB;
+  if (!encode_2d_bf16(&tmA, a.h, static_cast<uint64_t>(s.d), static_cast<uint64_t>(R), kBlockK, kBlockM))
+    return DG_ERR_CUDA;
+  if (!encode_2d_bf16(&tmB, a.E, static_cast<uint64_t>(s.d), static_cast<uint64_t>(s.V), kBlockK, kBlockN))
+    return DG_ERR_CUDA;
+
+  HeadParams hp;
+  memset(&hp, 0, sizeof(hp));
+  hp.R = R;
+  hp.d = s.d;
+  hp.V = s.V;
+  hp.B = s.B;
+  hp.split = head_split(R, s.V, s.d, sms);
+  hp.seed_lo = static_cast<uint32_t>(pr.seed & 0xFFFFFFFFull);
+  hp.seed_hi = static_cast<uint32_t>(pr.seed >> 32);
+  hp.e_scale = a.e_scale;
+  hp.part = reinterpret_cast<float*>(wsb + ws.part_off);
+  hp.err = reinterpret_cast<uint32_t*>(wsb + ws.err_off);
+  hp.logits_out = a.logits;
+  hp.wait_ns = kDefaultWaitNs;
+  memcpy(hp.cp, cps, sizeof(cps));
+
+  if (launch_head(tmA, tmB, hp, a.stream) != cudaSuccess) return DG_ERR_CUDA;
+
+  MergeParams mp;
+  memset(&mp, 0, sizeof(mp));
+  mp.R = R;
+  mp.B = s.B;
+  mp.V = s.V;
+  mp.P = ws.P;
+  mp.part = hp.part;
+  mp.entropy = a.entropy;
+  mp.sampled = a.sampled;
+  mp.argmax = a.argmax;
+  mp.canvas = a.canvas;
+  mp.prev_argmax = a.prev_argmax;
+  mp.accept = a.accept;
+  mp.stop = a.stop;
+  mp.tickets = reinterpret_cast<uint32_t*>(wsb + ws.tickets_off);
+  mp.seed_lo = hp.seed_lo;
+  mp.seed_hi = hp.seed_hi;
+  mp.entropy_bound = pr.entropy_bound;
+  mp.stop_entropy = pr.stop_entropy;
+  memcpy(mp.cp, cps, sizeof(cps));
+  if (launch_merge(mp, a.stream) != cudaSuccess) return DG_ERR_CUDA;
+  return DG_OK;
+}
+
+}  // namespace
+
+WsLayout ws_layout(const dg_shape& s, int num_sms) {
+  WsLayout w;
+  const int R = s.B * s.L;
+  const HeadSplit sp = head_split(R, s.V, s.d, num_sms);
+  w.P = 2 * sp.Q;
+  w.err_off = 0;
+  w.tickets_off = kAlign;
+  w.part_off = align_up(w.tickets_off + sizeof(uint32_t) * static_cast<size_t>(s.B));
+  w.total = align_up(w.part_off + sizeof(float) * kPartialFields * static_cast<size_t>(w.P) * R);
+  return w;
+}
+
+}  // namespace dg
+
+using namespace dg;
+
+extern "C" {
+
+dg_params dg_default_params(void) {
+  dg_params p;
+  p.tau0 = 0.8;
+  p.tau1 = 0.4;
+  p.max_steps = 48;
+  p.entropy_bound = 0.1;
+  p.stop_entropy = 0.005;
+  p.seed = 1234;
+  return p;
+}
+
+const char* dg_error_string(dg_status s) {
+  switch (s) {
+    case DG_OK: return "ok";
+    case DG_ERR_INVALID_ARG: return "invalid argument";
+    case DG_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case DG_ERR_WORKSPACE: return "workspace too small";
+    case DG_ERR_RANGE: return "step index out of range";
+    case DG_ERR_CUDA: return "CUDA runtime error";
+    case DG_ERR_TIMEOUT: return "device-side wait timed out";
+    case DG_ERR_CALLBACK: return "hidden-state callback failed";
+    case DG_ERR_NO_DEVICE: return "no sm_100 device";
+  }
+  return "unknown status";
+}
+
+size_t dg_workspace_size(const dg_shape* shape) {
+  if (check_shape(shape) != DG_OK) return 0;
+  const int sms = device_sms();
+  if (sms <= 0) return 0;
+  return ws_layout(*shape, sms).total;
+}
+
+dg_status dg_workspace_init(void* workspace, size_t ws_bytes, void* stream) {
+  if (workspace == nullptr) return DG_ERR_INVALID_ARG;
+  if (cudaMemsetAsync(workspace, 0, ws_bytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DG_ERR_CUDA;
+  return DG_OK;
+}
+
+dg_status dg_denoise_step(const dg_shape* shape, const dg_params* params, const void* h, const void* E,
+                          const float* e_scale, const int32_t* step_idx, const uint8_t* has_prev,
+                          const uint8_t* active, int32_t* canvas, int32_t* prev_argmax, uint8_t* accept,
+                          float* entropy, int32_t* sampled, int32_t* argmax, int32_t* stop,
+                          void* workspace, size_t ws_bytes, void* stream) {
+  StepArgs a{shape,   params,  h,      E,    e_scale, step_idx, has_prev, active,   canvas, prev_argmax,
+             accept,  entropy, sampled, argmax, stop,   nullptr,  workspace, ws_bytes,
+             static_cast<cudaStream_t>(stream)};
+  return run_step(a);
+}
+
+dg_status dg_debug_logits(const dg_shape* shape, const dg_params* params, const void* h, const void* E,
+                          const float* e_scale, const int32_t* step_idx, const uint8_t* has_prev,
+                          const uint8_t* active, int32_t* canvas, int32_t* prev_argmax, uint8_t* accept,
+                          float* entropy, int32_t* sampled, int32_t* argmax, int32_t* stop,
+                          float* logits, void* workspace, size_t ws_bytes, void* stream) {
+  if (logits == nullptr) return DG_ERR_INVALID_ARG;
+  StepArgs a{shape,   params,  h,      E,    e_scale, step_idx, has_prev, active,   canvas, prev_argmax,
+             accept,  entropy, sampled, argmax, stop,   logits,   workspace, ws_bytes,
+             static_cast<cudaStream_t>(stream)};
+  return run_step(a);
+}
+
+dg_status dg_device_status(void* workspace, size_t ws_bytes, void* stream) {
+  if (workspace == nullptr || ws_bytes < kAlign) return DG_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t err = 0;
+  if (cudaMemcpyAsync(&err, workspace, sizeof(err), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return DG_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return DG_ERR_CUDA;
+  if (err != 0) {
+    if (cudaMemsetAsync(workspace, 0, sizeof(err), st) != cudaSuccess) return DG_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return DG_ERR_CUDA;
+    return DG_ERR_TIMEOUT;
+  }
+  return DG_OK;
+}
+
+dg_status dg_denoise_loop(const dg_shape* shape, const dg_params* params, const void* E,
+                          const float* e_scale, dg_hidden_fn hidden_fn, void* user, int32_t k_start,
+                          void* h_buf, int32_t* canvas, int32_t* prev_argmax, uint8_t* has_prev,
+                          int32_t* steps_taken, uint8_t* accept, float* entropy, int32_t* sampled,
+                          int32_t* argmax, int32_t* stop, void* workspace, size_t ws_bytes,
+                          void* stream) {
+  dg_status st = check_shape(shape);
+  if (st != DG_OK) return st;
+  if ((st = check_params(params)) != DG_OK) return st;
+  if (hidden_fn == nullptr || h_buf == nullptr || has_prev == nullptr || steps_taken == nullptr)
+    return DG_ERR_INVALID_ARG;
+  if (k_start < 0 || k_start >= params->max_steps) return DG_ERR_RANGE;
+  const int B = shape->B, L = shape->L;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  int32_t ks[DG_MAX_B];
+  uint8_t act[DG_MAX_B];
+  int32_t stop_h[DG_MAX_B];
+  for (int b = 0; b < B; ++b) {
+    act[b] = 1;
+    steps_taken[b] = 0;
+  }
+  for (int k = k_start; k < params->max_steps; ++k) {
+    if (hidden_fn(k, canvas, h_buf, user, stream) != 0) return DG_ERR_CALLBACK;
+    for (int b = 0; b < B; ++b) ks[b] = k;
+    st = dg_denoise_step(shape, params, h_buf, E, e_scale, ks, has_prev, act, canvas, prev_argmax, accept,
+                         entropy, sampled, argmax, stop, workspace, ws_bytes, stream);
+    if (st != DG_OK) return st;
+    if (cudaMemcpyAsync(stop_h, stop, sizeof(int32_t) * B, cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+      return DG_ERR_CUDA;
+    if ((st = dg_device_status(workspace, ws_bytes, stream)) != DG_OK) return st;
+    bool any = false;
+    for (int b = 0; b < B; ++b) {
+      if (!act[b]) continue;
+      has_prev[b] = 1;
+      if (stop_h[b] || k == params->max_steps - 1) {
+        // commit: every slot takes this step's sampled token
+        if (cudaMemcpyAsync(canvas + static_cast<size_t>(b) * L, sampled + static_cast<size_t>(b) * L,
+                            sizeof(int32_t) * L, cudaMemcpyDeviceToDevice, cs) != cudaSuccess)
+          return DG_ERR_CUDA;
+        act[b] = 0;
+        steps_taken[b] = k - k_start + 1;
+      } else {
+        any = true;
+      }
+    }
+    if (!any) break;
+  }
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return DG_ERR_CUDA;
+  return DG_OK;
+}
+
+dg_status dg_selftest_bounded_wait(uint64_t limit_ns, void* workspace, size_t ws_bytes, void* stream) {
+  if (workspace == nullptr || ws_bytes < kAlign) return DG_ERR_INVALID_ARG;
+  if (device_sms() <= 0) return DG_ERR_NO_DEVICE;
+  if (launch_wait_selftest(static_cast<uint32_t*>(workspace), limit_ns, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return DG_ERR_CUDA;
+  return dg_device_status(workspace, ws_bytes, stream);
+}
+
+dg_status dg_debug_gumbel(const uint32_t* words, int32_t n, float* g_exact, float* lg2e_approx,
+                          void* stream) {
+  if (n < 0 || (n > 0 && (!words || !g_exact || !lg2e_approx))) return DG_ERR_INVALID_ARG;
+  if (device_sms() <= 0) return DG_ERR_NO_DEVICE;
+  if (launch_gumbel_probe(words, n, g_exact, lg2e_approx, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DG_ERR_CUDA;
+  return DG_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,313 @@
+// dg_device.cuh -- device building blocks of the sm_100a denoising step:
+// inline-PTX wrappers (mbarrier, TMA, tcgen05), Philox4x32-10, the
+// IEEE-only float32 log that defines the sampler's Gumbel key, and the fast
+// approximate key used to screen candidates.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#define DG_DEV __device__ __forceinline__
+
+namespace dg {
+
+// ---------------------------------------------------------------------------
+// status latch (shared with the host through the workspace)
+// ---------------------------------------------------------------------------
+enum : uint32_t {
+  kErrWaitTmaProducer = 1u << 0,  // producer gave up waiting for a free stage
+  kErrWaitMmaFull = 1u << 1,      // MMA issuer gave up waiting for a loaded stage
+  kErrWaitMmaAcc = 1u << 2,       // MMA issuer gave up waiting for a drained accumulator
+  kErrWaitEpilogue = 1u << 3,     // epilogue gave up waiting for a finished tile
+  kErrSelftest = 1u << 4,         // the bounded-wait self test ran out (expected)
+};
+
+// ---------------------------------------------------------------------------
+// small PTX helpers
+// ---------------------------------------------------------------------------
+DG_DEV uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+DG_DEV uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+DG_DEV void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+DG_DEV void fence_mbarrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+DG_DEV void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+DG_DEV void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
+               "r"(bytes)
+               : "memory");
+}
+
+DG_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for the phase of parity `parity` to complete, for at most `limit_ns`
+// nanoseconds of %globaltimer.  Returns false if the limit ran out.
+DG_DEV bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (global_timer_ns() - t0 > limit_ns) return false;
+  }
+}
+
+// 2-D tiled TMA load into this CTA's shared memory, completing on `bar`.
+// x is the inner (contiguous) coordinate in elements, y the row.
+DG_DEV void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y,
+                        uint64_t cache_hint) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "l"(cache_hint)
+      : "memory");
+}
+
+DG_DEV void prefetch_tensormap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// L2 cache-policy words for the TMA cache hint.
+DG_DEV uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+DG_DEV uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// ---------------------------------------------------------------------------
+// tcgen05 (5th-generation tensor core, accumulators in tensor memory)
+// ---------------------------------------------------------------------------
+DG_DEV void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+}
+DG_DEV void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+DG_DEV void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+DG_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+DG_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Arrive once on `bar` when every tcgen05 operation issued so far by this
+// thread has completed.
+DG_DEV void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, f32 accumulate.
+DG_DEV void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major tile stored by TMA with the
+// 128-byte swizzle: rows of 128 B, 8-row (1024 B) swizzle atoms stacked
+// along M/N.  Fields: start address >> 4 [0,14), leading byte offset >> 4
+// [16,30) (unused by swizzled K-major, set to 1), stride byte offset >> 4
+// [32,46) = 1024 B between 8-row groups, descriptor version 1 at [46,48),
+// base offset 0 (tiles are 1024-B aligned), swizzle mode 2 (128 B) at [61,64).
+DG_DEV uint64_t smem_desc_k_sw128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(1u) << 16;
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
+// Instruction descriptor, kind::f16: f32 accumulator [4,6)=1, A bf16
+// [7,10)=1, B bf16 [10,13)=1, both K-major (bits 15, 16 = 0), N>>3 at
+// [17,23), M>>4 at [24,29).
+__host__ __device__ constexpr uint32_t instr_desc_bf16_f32(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// 32 consecutive f32 columns of this thread's TMEM lane (32x32b shape), with
+// the wait folded into the same statement so no use can move above it.
+DG_DEV void tmem_load_32cols(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ---------------------------------------------------------------------------
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11): ten rounds of
+// (x0,x1,x2,x3) -> (hi(M1 x2)^x1^k0, lo(M1 x2), hi(M0 x0)^x3^k1, lo(M0 x0))
+// with the key bumped by the Weyl constants after each round.
+// ---------------------------------------------------------------------------
+DG_DEV void philox4x32_10(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3, uint32_t k0,
+                          uint32_t k1, uint32_t (&out)[4]) {
+#pragma unroll
+  for (int i = 0; i < 10; ++i) {
+    const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * x0;
+    const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * x2;
+    const uint32_t y0 = static_cast<uint32_t>(p1 >> 32) ^ x1 ^ k0;
+    const uint32_t y2 = static_cast<uint32_t>(p0 >> 32) ^ x3 ^ k1;
+    x1 = static_cast<uint32_t>(p1);
+    x3 = static_cast<uint32_t>(p0);
+    x0 = y0;
+    x2 = y2;
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  out[0] = x0;
+  out[1] = x1;
+  out[2] = x2;
+  out[3] = x3;
+}
+
+// Stream purposes (high half of counter word 1).
+constexpr uint32_t kPurposeGumbel = 0u;
+constexpr uint32_t kPurposeRenoise = 1u;
+
+// ---------------------------------------------------------------------------
+// The float32 key of the Gumbel-max draw, IEEE operations only.
+//
+// L(y): y = 2^e m, m in [1,2), halved (e+1) when m > sqrt(2); f = m - 1,
+// s = f / (m + 1), z = s^2, ln m = 2s + s z (2/3 + z (2/5 + z (2/7 + z (2/9
+// + z 2/11)))) (the atanh series of ln m = 2 atanh((m-1)/(m+1))), result
+// e LN2_HI + (ln m + e LN2_LO) with LN2_HI = ln 2 truncated to 16 fraction
+// bits.  Every constant is the float32 nearest to the stated rational.
+// ---------------------------------------------------------------------------
+DG_DEV float log_ieee(float y) {
+  const float kC3 = __uint_as_float(0x3f2aaaabu);   // RN(2/3)
+  const float kC5 = __uint_as_float(0x3ecccccdu);   // RN(2/5)
+  const float kC7 = __uint_as_float(0x3e924925u);   // RN(2/7)
+  const float kC9 = __uint_as_float(0x3e638e39u);   // RN(2/9)
+  const float kC11 = __uint_as_float(0x3e3a2e8cu);  // RN(2/11)
+  const float kLn2Hi = __uint_as_float(0x3f317200u);  // 45426 / 65536
+  const float kLn2Lo = __uint_as_float(0x35bfbe8eu);  // RN(ln 2 - LN2_HI)
+  const uint32_t b = __float_as_uint(y);
+  int e = static_cast<int>((b >> 23) & 0xFFu) - 127;
+  const uint32_t mant = b & 0x7FFFFFu;
+  float m = __uint_as_float(mant | 0x3F800000u);
+  if (mant > 0x3504F3u) {  // m > sqrt(2)
+    m = __fmul_rn(m, 0.5f);
+    e += 1;
+  }
+  const float f = __fsub_rn(m, 1.0f);
+  const float s = __fdiv_rn(f, __fadd_rn(m, 1.0f));
+  const float z = __fmul_rn(s, s);
+  float r = __fmul_rn(z, kC11);
+  r = __fadd_rn(kC9, r);
+  r = __fmul_rn(z, r);
+  r = __fadd_rn(kC7, r);
+  r = __fmul_rn(z, r);
+  r = __fadd_rn(kC5, r);
+  r = __fmul_rn(z, r);
+  r = __fadd_rn(kC3, r);
+  r = __fmul_rn(z, r);
+  const float lnm = __fadd_rn(__fadd_rn(s, s), __fmul_rn(s, r));
+  const float ef = static_cast<float>(e);
+  return __fadd_rn(__fmul_rn(ef, kLn2Hi), __fadd_rn(lnm, __fmul_rn(ef, kLn2Lo)));
+}
+
+// u = (2 (r >> 9) + 1) 2^-24, exact.
+DG_DEV float uniform_from_word(uint32_t r) {
+  return __fmul_rn(static_cast<float>(2u * (r >> 9) + 1u), 5.9604644775390625e-08f);
+}
+
+// g32(u) = -L(-L(u)): the Gumbel noise of the specified key.
+DG_DEV float gumbel_exact(uint32_t r) {
+  const float u = uniform_from_word(r);
+  return -log_ieee(-log_ieee(u));
+}
+
+// The specified float32 key: fl(fl(z * inv_tau) + g32).
+DG_DEV float key_exact(float z, float inv_tau, uint32_t r) {
+  return __fadd_rn(__fmul_rn(z, inv_tau), gumbel_exact(r));
+}
+
+DG_DEV float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+DG_DEV float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// log2 of the Exp(1) variable E = -ln u, approximately.  For u > 15/16
+// (y = 1 - u < 1/16, where lg2 of u loses relative accuracy) E comes from
+// -ln(1 - y) = y (1 + y/2 + y^2/3 + y^3/4 + ...); otherwise from the fast
+// hardware log2.  Returns lg2(E) so that g = -ln 2 * lg2(E).  The result's
+// distance from the exact transform is measured over all 2^23 inputs by the
+// GPU tests and bounded by kGumbelApproxErr.
+DG_DEV float lg2_exp1_approx(uint32_t r) {
+  const float one_plus = __uint_as_float((r >> 9) | 0x3F800000u);  // 1 + r23 2^-23
+  const float u = __fsub_rn(one_plus, __uint_as_float(0x3f7fffffu));  // - (1 - 2^-24), exact
+  const float y = __fsub_rn(1.0f, u);                                 // exact
+  float t = __fmaf_rn(y, 0.25f, __uint_as_float(0x3eaaaaabu));        // 1/3 + y/4
+  t = __fmaf_rn(y, t, 0.5f);
+  t = __fmaf_rn(y, t, 1.0f);
+  const float e_series = __fmul_rn(y, t);
+  const float e_log = __fmul_rn(lg2_approx(u), -0.693147182464599609375f);
+  const float e = (y < 0.0625f) ? e_series : e_log;
+  return lg2_approx(e);
+}
+
+// |approx key - specified key| <= kGumbelApproxErr + rounding of the keys.
+constexpr float kGumbelApproxErr = 1.0e-5f;
+constexpr float kLn2 = 0.693147182464599609375f;
+constexpr float kLog2e = 1.44269502162933349609375f;
+
+}  // namespace dg

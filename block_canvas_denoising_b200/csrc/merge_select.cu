@@ -1,0 +1,188 @@
+// merge_select.cu -- cross-tile merge of the head's partials, then the
+// per-canvas entropy-bounded selection, renoise and stop test.
+//
+// Each CTA merges the partial records of 32 rows (8 threads per row, fixed
+// order), writes entropy / sampled / argmax of those rows and takes a ticket
+// on its canvas; the CTA that takes the last ticket of a canvas runs the
+// per-canvas step for all 256 slots:
+//   * selection ([Docs] "DiffusionGemma", Recommended serving configuration,
+//     token selection, entropy bound 0.1): slots ordered by (entropy, slot);
+//     slot s is accepted when the running entropy sum up to and including s
+//     is <= the bound, and the lowest-entropy slot always is;
+//   * renoise (same row: unselected tokens fully renoised; [Report]
+//     "DiffusionGemma Technical Report", Figure 3: uniform noise): token
+//     (r V) >> 32 from Philox counter (0, slot | 1 << 16, k, b), lane 0;
+//   * stop ([Docs] adaptive early stopping, threshold 0.005): the canvas
+//     has a previous prediction, its mean entropy is below the threshold and
+//     every slot's argmax equals the previous one.
+#include <float.h>
+#include <limits.h>
+
+#include "dg_device.cuh"
+#include "dg_internal.h"
+
+namespace dg {
+
+namespace {
+
+constexpr int kRowsPerCta = 32;
+constexpr int kPartsPerRow = 8;
+
+struct Acc {
+  float m2, S, T2, zmax;
+  int zarg;
+  float gkey;
+  int garg;
+};
+
+DG_DEV void acc_init(Acc& a) {
+  a.m2 = -1.0e30f;
+  a.S = 0.f;
+  a.T2 = 0.f;
+  a.zmax = -FLT_MAX;
+  a.zarg = INT_MAX;
+  a.gkey = -FLT_MAX;
+  a.garg = INT_MAX;
+}
+
+// Merge b into a.  Softmax: m = max(m_a, m_b), S = sum_i S_i 2^(m_i - m),
+// T2 = sum_i (T2_i + (m_i - m) S_i) 2^(m_i - m).  Argmax and Gumbel key: the
+// larger value wins, ties to the lower vocabulary index.
+DG_DEV void acc_merge(Acc& a, const Acc& b) {
+  const float m = fmaxf(a.m2, b.m2);
+  const float da = a.m2 - m, db = b.m2 - m;
+  const float sa = exp2f(da), sb = exp2f(db);
+  a.T2 = (a.T2 + da * a.S) * sa + (b.T2 + db * b.S) * sb;
+  a.S = a.S * sa + b.S * sb;
+  a.m2 = m;
+  if (b.zmax > a.zmax || (b.zmax == a.zmax && b.zarg < a.zarg)) {
+    a.zmax = b.zmax;
+    a.zarg = b.zarg;
+  }
+  if (b.gkey > a.gkey || (b.gkey == a.gkey && b.garg < a.garg)) {
+    a.gkey = b.gkey;
+    a.garg = b.garg;
+  }
+}
+
+DG_DEV Acc acc_load(const float* part, size_t plane, size_t idx) {
+  Acc a;
+  a.m2 = __ldcg(part + 0 * plane + idx);
+  a.S = __ldcg(part + 1 * plane + idx);
+  a.T2 = __ldcg(part + 2 * plane + idx);
+  a.zmax = __ldcg(part + 3 * plane + idx);
+  a.zarg = __float_as_int(__ldcg(part + 4 * plane + idx));
+  a.gkey = __ldcg(part + 5 * plane + idx);
+  a.garg = __float_as_int(__ldcg(part + 6 * plane + idx));
+  return a;
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(256)
+merge_select_kernel(const __grid_constant__ MergeParams p) {
+  __shared__ Acc s_acc[kPartsPerRow][kRowsPerCta];
+  __shared__ unsigned long long s_key[256];
+  __shared__ float s_h[256];
+  __shared__ double s_red[8];
+  __shared__ int s_last;
+
+  const int t = threadIdx.x;
+  const int r_local = t & (kRowsPerCta - 1);
+  const int part_id = t >> 5;
+  const int row = blockIdx.x * kRowsPerCta + r_local;
+  const size_t plane = static_cast<size_t>(p.P) * p.R;
+
+  // ---- merge partials of this row: thread part_id takes p = part_id, +8, ...
+  Acc a;
+  acc_init(a);
+  for (int q = part_id; q < p.P; q += kPartsPerRow)
+    acc_merge(a, acc_load(p.part, plane, static_cast<size_t>(q) * p.R + row));
+  s_acc[part_id][r_local] = a;
+  __syncthreads();
+  if (part_id == 0) {
+#pragma unroll
+    for (int i = 1; i < kPartsPerRow; ++i) acc_merge(a, s_acc[i][r_local]);
+    // H = ln S - ln2 T2 / S, clamped at 0 (the exact value is >= 0)
+    float H = logf(a.S) - kLn2 * a.T2 / a.S;
+    H = fmaxf(H, 0.0f);
+    p.entropy[row] = H;
+    p.sampled[row] = a.garg;
+    p.argmax[row] = a.zarg;
+  }
+
+  // ---- ticket: the last CTA of this canvas does the per-canvas step
+  const int b = (blockIdx.x * kRowsPerCta) >> 8;
+  __threadfence();
+  __syncthreads();
+  if (t == 0) {
+    const uint32_t ctas_per_canvas = 256 / kRowsPerCta;
+    const uint32_t prev = atomicAdd(&p.tickets[b], 1u);
+    s_last = (prev == ctas_per_canvas - 1) ? 1 : 0;
+    if (s_last) p.tickets[b] = 0u;  // reset for the next step
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+
+  const CanvasParam cp = p.cp[b];
+  const int s = t;  // slot
+  const int grow = b * 256 + s;
+  const float H = __ldcg(p.entropy + grow);
+  const int samp = __ldcg(p.sampled + grow);
+  const int amax = __ldcg(p.argmax + grow);
+
+  // ---- entropy-bounded selection: order by (H, slot); H >= 0 so its bits
+  // order like the values
+  const unsigned long long key =
+      (static_cast<unsigned long long>(__float_as_uint(H)) << 32) | static_cast<unsigned>(s);
+  s_key[s] = key;
+  s_h[s] = H;
+  __syncthreads();
+  double csum = 0.0;
+  int rank = 0;
+#pragma unroll 8
+  for (int i = 0; i < 256; ++i) {
+    const unsigned long long ki = s_key[i];
+    if (ki <= key) csum += static_cast<double>(s_h[i]);
+    rank += (ki < key) ? 1 : 0;
+  }
+  const bool accepted = (csum <= p.entropy_bound) || (rank == 0);
+
+  // ---- renoise
+  int tok = samp;
+  if (!accepted) {
+    uint32_t r[4];
+    philox4x32_10(0u, static_cast<uint32_t>(s) | (kPurposeRenoise << 16), static_cast<uint32_t>(cp.k),
+                  static_cast<uint32_t>(b), p.seed_lo, p.seed_hi, r);
+    tok = static_cast<int>((static_cast<uint64_t>(r[0]) * static_cast<uint64_t>(p.V)) >> 32);
+  }
+
+  // ---- stop: mean entropy (float64 sum in a fixed tree order) and agreement
+  double hsum = static_cast<double>(H);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) hsum += __shfl_xor_sync(0xffffffffu, hsum, off);
+  if ((t & 31) == 0) s_red[t >> 5] = hsum;
+  const int prev = cp.active ? p.prev_argmax[grow] : amax;
+  const int same = __syncthreads_and(prev == amax);
+  double total = 0.0;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) total += s_red[w];
+  const double mean_h = total / 256.0;
+  const bool stop = cp.has_prev && same && (mean_h < p.stop_entropy);
+
+  if (cp.active) {
+    p.accept[grow] = accepted ? 1 : 0;
+    p.canvas[grow] = tok;
+    p.prev_argmax[grow] = amax;
+    if (t == 0) p.stop[b] = stop ? 1 : 0;
+  }
+}
+
+cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream) {
+  const int grid = p.R / kRowsPerCta;
+  merge_select_kernel<<<grid, 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace dg

@@ -1,0 +1,207 @@
+/*
+ * dg.h -- C ABI of the B200 denoising-step library (libdg.so).
+ *
+ * One denoising step of block discrete-diffusion text generation over
+ * canvases of L = 256 token slots: the tied LM head z = h . E^T fused with
+ * the sampler (temperature-scaled softmax entropy, Gumbel-max draw),
+ * entropy-bounded acceptance, full renoise of the unaccepted slots and the
+ * adaptive-stop test.  Sources, by page title and section:
+ *
+ *   [Docs]   "DiffusionGemma" (Google AI for Developers model docs), table
+ *            "Recommended serving configuration": max 48 denoising steps,
+ *            temperature linear 0.8 -> 0.4, adaptive stop at mean entropy
+ *            0.005 with two identical consecutive predictions, token
+ *            selection with entropy bound 0.1 and full renoise of the rest.
+ *   [Report] "DiffusionGemma Technical Report" (arXiv:2608.00146), Table 1
+ *            (262k vocabulary, 740M embedder => d = 2816), Figure 3 (uniform
+ *            noise), Figure 4 (denoising loop over a 256-token canvas).
+ *   [Press]  "Google DiffusionGemma generates 256 tokens in parallel and
+ *            self-corrects", section "What DiffusionGemma does" (every
+ *            position re-evaluated each step; low-confidence positions are
+ *            randomised; the settled block's remaining tokens are locked).
+ *
+ * Conventions for every entry point:
+ *   - Tensors are DEVICE pointers owned by the caller unless marked "host".
+ *     The library allocates no device memory; scratch lives in a caller
+ *     workspace of dg_workspace_size() bytes, zeroed once by
+ *     dg_workspace_init() before its first use.
+ *   - Row r = b*L + s of a [B*L, ...] tensor is slot s of canvas b.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t, NULL =
+ *     legacy default stream).  Argument errors are detected on the host
+ *     before anything is launched.  Faults detected on the device (a
+ *     bounded wait that ran out) are latched in the workspace and reported
+ *     by dg_device_status().
+ *   - Errors are returned, never raised: no exit(), no abort().
+ *   - Calls that share a workspace must not overlap on the device.
+ */
+#ifndef DG_H
+#define DG_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DG_OK = 0,
+  DG_ERR_INVALID_ARG = 1,      /* null pointer, misalignment, bad parameter */
+  DG_ERR_UNSUPPORTED_SHAPE = 2,/* L != 256, d % 64, V % 256, B out of range */
+  DG_ERR_WORKSPACE = 3,        /* workspace smaller than dg_workspace_size() */
+  DG_ERR_RANGE = 4,            /* a step index k outside [0, max_steps) */
+  DG_ERR_CUDA = 5,             /* a CUDA runtime call failed */
+  DG_ERR_TIMEOUT = 6,          /* a device-side bounded wait ran out */
+  DG_ERR_CALLBACK = 7,         /* the hidden-state callback returned non-zero */
+  DG_ERR_NO_DEVICE = 8         /* no sm_100 device current */
+} dg_status;
+
+typedef enum { DG_E_BF16 = 0, DG_E_FP8_E4M3 = 1 } dg_edtype;
+
+/* Problem shape.  L must be 256 ([Report] Figure 4: 256-token canvas);
+ * d a multiple of 64 and >= 64; V a multiple of 256 and >= 256;
+ * 1 <= B <= DG_MAX_B. */
+typedef struct {
+  int32_t B;        /* canvases per step */
+  int32_t L;        /* slots per canvas (256) */
+  int32_t d;        /* hidden size */
+  int32_t V;        /* vocabulary size */
+  int32_t e_dtype;  /* dg_edtype of the embedder */
+} dg_shape;
+
+#define DG_MAX_B 256
+
+/* Sampler parameters; dg_default_params() gives the [Docs] serving
+ * defaults (tau0 0.8, tau1 0.4, 48 steps, bound 0.1, stop 0.005). */
+typedef struct {
+  double tau0;           /* temperature at step 0 */
+  double tau1;           /* temperature at step max_steps-1 */
+  int32_t max_steps;     /* N, at most this many steps per canvas */
+  double entropy_bound;  /* selection bound on the cumulative entropy */
+  double stop_entropy;   /* adaptive stop: canvas-mean entropy threshold */
+  uint64_t seed;         /* Philox4x32-10 key (low word, high word) */
+} dg_params;
+
+dg_params dg_default_params(void);
+
+/* Human-readable name of a status code (static storage). */
+const char* dg_error_string(dg_status s);
+
+/* Bytes of device workspace one step of this shape needs on the current
+ * device (it depends on the device's SM count).  Returns 0 for an invalid
+ * shape. */
+size_t dg_workspace_size(const dg_shape* shape);
+
+/* Zero a workspace (enqueued on `stream`).  Needed once per workspace. */
+dg_status dg_workspace_init(void* workspace, size_t ws_bytes, void* stream);
+
+/* dg_denoise_step -- one denoising step of B canvases.
+ *
+ * Inputs
+ *   h         bf16 [B*L, d] row-major: canvas hidden states.
+ *   E         embedder [V, d] row-major: bf16, or FP8-E4M3 codes (uint8)
+ *             when shape->e_dtype == DG_E_FP8_E4M3.  The tied LM head
+ *             ([Report] Table 1) is z = h . E^T (times e_scale[v] for FP8).
+ *   e_scale   float [V] per-row dequantisation scale (FP8 only, else NULL).
+ *   step_idx  HOST int32 [B]: step k of each canvas, 0 <= k < max_steps.
+ *             tau_k = tau0 - (tau0 - tau1) * k / (max_steps - 1)
+ *             ([Docs] temperature schedule), tau0 for max_steps == 1.
+ *   has_prev  HOST uint8 [B]: 1 if prev_argmax holds the previous step's
+ *             prediction for that canvas (0 on a canvas's first step).
+ *   active    HOST uint8 [B] or NULL (= all 1): canvases with 0 are left
+ *             untouched (canvas, prev_argmax, accept, stop not written).
+ * In/out
+ *   canvas      int32 [B*L]: overwritten with the new canvas (accepted slots
+ *               take the sampled token, the rest a uniform random token).
+ *   prev_argmax int32 [B*L]: read as the previous prediction, then
+ *               overwritten with this step's argmax prediction.
+ * Outputs
+ *   accept   uint8 [B*L]   entropy-bounded acceptance mask.
+ *   entropy  float [B*L]   entropy (nats) of softmax(z / tau_k).
+ *   sampled  int32 [B*L]   Gumbel-max draw from softmax(z / tau_k).
+ *   argmax   int32 [B*L]   argmax_v z (ties to the lower v).
+ *   stop     int32 [B]     adaptive-stop flag of each canvas.
+ * Scratch
+ *   workspace, ws_bytes >= dg_workspace_size(shape), zeroed once.
+ * h and E must be 16-byte aligned.  Asynchronous on `stream`.
+ */
+dg_status dg_denoise_step(const dg_shape* shape, const dg_params* params,
+                          const void* h, const void* E, const float* e_scale,
+                          const int32_t* step_idx, const uint8_t* has_prev,
+                          const uint8_t* active,
+                          int32_t* canvas, int32_t* prev_argmax,
+                          uint8_t* accept, float* entropy, int32_t* sampled,
+                          int32_t* argmax, int32_t* stop,
+                          void* workspace, size_t ws_bytes, void* stream);
+
+/* dg_debug_logits -- the same step as dg_denoise_step (same kernels, same
+ * outputs) that also writes the raw float32 logits z [B*L, V] the fused
+ * sampler consumed.  For parity checks only: it writes B*L*V*4 bytes. */
+dg_status dg_debug_logits(const dg_shape* shape, const dg_params* params,
+                          const void* h, const void* E, const float* e_scale,
+                          const int32_t* step_idx, const uint8_t* has_prev,
+                          const uint8_t* active,
+                          int32_t* canvas, int32_t* prev_argmax,
+                          uint8_t* accept, float* entropy, int32_t* sampled,
+                          int32_t* argmax, int32_t* stop, float* logits,
+                          void* workspace, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, then read and clear the device fault latch of the
+ * workspace.  Returns DG_OK, DG_ERR_TIMEOUT or DG_ERR_CUDA. */
+dg_status dg_device_status(void* workspace, size_t ws_bytes, void* stream);
+
+/* Hidden-state producer for the loop: writes the bf16 [B*L, d] hidden
+ * states of step k for the current canvas into h_out (device), enqueued on
+ * `stream`.  Returns 0 on success; anything else stops the loop with
+ * DG_ERR_CALLBACK.  It stands in for the denoiser's forward pass. */
+typedef int (*dg_hidden_fn)(int32_t k, const int32_t* canvas, void* h_out,
+                            void* user, void* stream);
+
+/* dg_denoise_loop -- the adaptive loop ([Docs] max steps and adaptive stop;
+ * [Report] Figure 4).  For k = k_start, k_start+1, ...: hidden_fn writes h,
+ * one dg_denoise_step runs on every still-active canvas, the B stop flags
+ * are read back (one device->host copy per step).  A canvas that stops, or
+ * reaches k = max_steps-1, commits: every slot takes that step's sampled
+ * token ([Press] "remaining tokens are locked") and the canvas is frozen.
+ *
+ *   h_buf        bf16 [B*L, d] device buffer handed to hidden_fn.
+ *   canvas       int32 [B*L] in/out: the committed canvas on return.
+ *   prev_argmax  int32 [B*L] in/out: prediction state (see has_prev).
+ *   has_prev     HOST uint8 [B] in/out: resume state; all 0 for a fresh start.
+ *   steps_taken  HOST int32 [B] out: steps run for each canvas.
+ *   accept, entropy, sampled, argmax, stop: device outputs of the last step.
+ * Resuming with the state of an interrupted loop at k_start gives the same
+ * result as the uninterrupted run (the random streams are counter-based).
+ */
+dg_status dg_denoise_loop(const dg_shape* shape, const dg_params* params,
+                          const void* E, const float* e_scale,
+                          dg_hidden_fn hidden_fn, void* user, int32_t k_start,
+                          void* h_buf, int32_t* canvas, int32_t* prev_argmax,
+                          uint8_t* has_prev, int32_t* steps_taken,
+                          uint8_t* accept, float* entropy, int32_t* sampled,
+                          int32_t* argmax, int32_t* stop,
+                          void* workspace, size_t ws_bytes, void* stream);
+
+/* ---- diagnostics (no counterpart on the pages; used by the tests) ---- */
+
+/* Self test of the device-side bounded wait: launches one kernel that waits
+ * on a barrier nothing ever arrives at, gives up after limit_ns
+ * nanoseconds, latches the fault in the workspace and returns normally.
+ * The call synchronises `stream` and returns DG_ERR_TIMEOUT when the wait
+ * ran out as designed (the context stays usable), DG_OK otherwise. */
+dg_status dg_selftest_bounded_wait(uint64_t limit_ns, void* workspace, size_t ws_bytes,
+                                   void* stream);
+
+/* For n Philox words (device uint32 [n]) write the specified float32
+ * Gumbel noise g32 = -L(-L(u)) (device float [n]) and the log2 of the
+ * approximate Exp(1) variable the sampler's screening pass uses (device
+ * float [n]), so tests can compare both with the oracle and bound the
+ * approximation over every possible input. */
+dg_status dg_debug_gumbel(const uint32_t* words, int32_t n, float* g_exact, float* lg2e_approx,
+                          void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DG_H */

@@ -1,0 +1,80 @@
+"""The C-ABI library loads and exports every entry point ``include/dg.h``
+declares; host-side argument checks answer without a device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import block_canvas_denoising_b200 as dg
+from block_canvas_denoising_b200 import build as dg_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "dg.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = set(re.findall(r"\b(dg_[a-z_0-9]+)\s*\(", text))
+    # typedef'd function pointer types are not exported symbols
+    names -= set(re.findall(r"\(\s*\*\s*(dg_[a-z_0-9]+)\s*\)", text))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def libdg():
+    dg_build.build()
+    return dg.lib()
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for required in ("dg_denoise_step", "dg_denoise_loop", "dg_workspace_size", "dg_debug_logits",
+                     "dg_error_string", "dg_device_status"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(libdg):
+    missing = [n for n in _declared() if not hasattr(libdg, n)]
+    assert not missing, missing
+
+
+def test_default_params_are_serving_defaults(libdg):
+    p = libdg.dg_default_params()
+    assert (p.tau0, p.tau1, p.max_steps, p.entropy_bound, p.stop_entropy) == (0.8, 0.4, 48, 0.1, 0.005)
+
+
+def test_error_strings(libdg):
+    for code in range(9):
+        assert libdg.dg_error_string(code)
+
+
+def _call_step(libdg, B=1, L=256, d=512, V=8192, ks=(0,), e_dtype=0, null=False):
+    shp = dg._Shape(B, L, d, V, e_dtype)
+    prm = dg.Params().c()
+    ksa = np.asarray(ks, np.int32)
+    hp = np.zeros(max(B, 1), np.uint8)
+    fake = ctypes.c_void_p(0 if null else 256)   # never dereferenced: checks fail first
+    P = [fake] * 9
+    return libdg.dg_denoise_step(ctypes.byref(shp), ctypes.byref(prm), fake, fake, None,
+                                 ksa.ctypes.data_as(ctypes.c_void_p), hp.ctypes.data_as(ctypes.c_void_p),
+                                 None, *P[:7], fake, ctypes.c_size_t(1 << 30), None)
+
+
+def test_shape_checks_before_any_device_work(libdg):
+    assert _call_step(libdg, L=128) == 2
+    assert _call_step(libdg, d=100) == 2
+    assert _call_step(libdg, V=1000) == 2
+    assert _call_step(libdg, B=0, ks=()) == 2
+    assert _call_step(libdg, B=257, ks=[0] * 257) == 2
+
+
+def test_null_and_range_checks(libdg):
+    assert _call_step(libdg, null=True) == 1
+    assert _call_step(libdg, ks=(48,)) == 4
+    assert _call_step(libdg, ks=(-1,)) == 4
+
+
+def test_workspace_size_zero_for_bad_shape(libdg):
+    assert dg.workspace_size(1, 100, 8192) == 0
