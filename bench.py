@@ -1,0 +1,430 @@
+#!/usr/bin/env python
+"""Benchmark of the denoising step on B200: prints ONE JSON line (rank 0).
+
+Workload: the production-shape step -- one 256-slot canvas per GPU (B=1),
+d = 2816, V = 262,144, bf16 hidden states and embedder (synthetic N(0,1)
+and N(0, 0.02^2), seeded), the step index cycling through k = 0, 23, 47
+(tau 0.8, 0.604, 0.4).  A "step" is one pass of the whole path: the fused
+tied-head + sampler kernel and the merge/selection/renoise/stop kernel.
+The embedder (1.48 GB) is far larger than the 126 MB L2, so every step
+streams it from HBM; no flush is needed.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+For N > 1 launch with torch.distributed.run; each rank runs its own canvas
+(replicas, no data-path collective): weak scaling.  ``--impl reference``
+times the CPU oracle (the only reference implementation there is) on the
+host cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("denoise-step µs & canvas slots/s at B=1, 256×2816×262144 bf16; "
+          "% of roofline")
+B, L, D, V = 1, 256, 2816, 262144
+KS = (0, 23, 47)
+REF_BUDGET_S = 90.0      # wall-clock cap of the oracle's timed steps
+SOAK_S = 1.0             # untimed steady-load run before the timed region
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+HEAD_SOURCES = ("block_canvas_denoising_b200/csrc/head_sampler.cu",
+                "block_canvas_denoising_b200/csrc/dg_device.cuh",
+                "block_canvas_denoising_b200/csrc/dg_internal.h")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def head_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in HEAD_SOURCES:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per launch of the fused kernel from the committed ncu
+    summary, if it was taken on the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "head_sampler_traffic.json")
+    if not os.path.exists(p):
+        return None, None
+    d = json.load(open(p))
+    if d.get("kernel_source_sha256_16") != head_source_hash():
+        return None, d.get("kernel_source_sha256_16")
+    return d.get("dram_bytes_per_launch"), d.get("kernel_source_sha256_16")
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 10:
+                    rows.append(parts[1:] + [parts[0]])
+            os.unlink(self.path)
+        return rows
+
+    @staticmethod
+    def within(rows, t0, t1):
+        """Rows whose timestamp (last field) lies in [t0, t1] (epoch s)."""
+        import datetime
+        out = []
+        for r in rows:
+            try:
+                ts = datetime.datetime.strptime(r[-1], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                continue
+            if t0 <= ts <= t1:
+                out.append(r)
+        return out
+
+    @staticmethod
+    def summarize(rows):
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip().lower() == "active"})
+        # samples while the GPU was busy (clock above idle) describe the load
+        busy = [s for s in sm if s > 600] or sm
+        return {"sm_mhz": statistics.median(busy) if busy else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(sm)}
+
+
+def bad_clocks(c) -> bool:
+    if any(r in c["reasons"] for r in ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")):
+        return True
+    if c["sm_mhz"] and c["sm_max_mhz"] and not c["reasons"] and c["sm_mhz"] < 0.5 * c["sm_max_mhz"]:
+        return True
+    return False
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample of the same workload)
+# ---------------------------------------------------------------------------
+def oracle_canvas_step(h_bits, E_bits, k):
+    import oracle
+    t0 = time.perf_counter()
+    oracle.denoise_step(h_bits, E_bits=E_bits, B=1, L=L, step_idx=np.array([k], np.int32),
+                        has_prev=np.zeros(1, np.uint8), prev_argmax=np.zeros(L, np.int32))
+    return time.perf_counter() - t0
+
+
+def oracle_rows_step(h_bits, E_bits, k, rows: int):
+    """The oracle's per-slot path (logits, entropy, argmax, Gumbel draw) on
+    ``rows`` slots plus its per-canvas selection / renoise / stop on them."""
+    from oracle import step as S
+    t0 = time.perf_counter()
+    tau = S.temperature(k)
+    z = S.logits(h_bits[:rows], E_bits=E_bits)
+    x = z / tau
+    H = S.entropy(x)
+    amax = S.argmax_lowest(z)
+    w = S.gumbel_words(np.arange(rows), 0, k, V, seed=1234)
+    samp, _ = S.gumbel_sample(x, w)
+    acc, _, _ = S.select(H)
+    noise = S.renoise_tokens(0, k, rows, V, 1234)
+    np.where(acc == 1, samp, noise)
+    S.stop_flag(H, amax, amax, False)
+    return time.perf_counter() - t0
+
+
+def threads_used() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------------------
+def init_dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_reference(args):
+    world, rank, _ = init_dist()
+    if world > 1 and rank != 0:
+        return 0
+    import synth
+    E = synth.embedder_normal(V, D, seed=1)
+    h = synth.hidden_normal(B, L, D, seed=2)
+    rows = 32
+    for i in range(max(0, min(args.warmup, 1))):
+        oracle_rows_step(h, E, KS[i % 3], rows)
+    # each oracle step costs seconds: time at most REF_BUDGET_S of them
+    times = []
+    t_start = time.perf_counter()
+    for i in range(args.steps):
+        times.append(oracle_rows_step(h, E, KS[i % 3], rows))
+        if time.perf_counter() - t_start > REF_BUDGET_S:
+            break
+    t = sum(times) / len(times)
+    val = rows / t
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "slots/s",
+        "n_gpus": args.gpus, "steps": len(times), "steps_requested": args.steps,
+        "warmup": args.warmup, "ms_per_step": t * 1e3 * (L / rows), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "B=1 canvas, L=256, d=2816, V=262144, bf16 inputs, k cycling 0/23/47",
+                   "global_batch": 1, "seq_len": L, "parallelism": "cpu oracle"},
+        "cpu_baseline": {"value": val, "unit": "slots/s", "cores": threads_used(), "kind": "oracle",
+                         "sample": f"{rows} of 256 slots per step (full vocabulary), "
+                                   "plus selection/renoise/stop on them"},
+        "e2e": {"value": val, "unit": "slots/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    world, rank, local = init_dist()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    import block_canvas_denoising_b200 as dg
+    import synth
+    from block_canvas_denoising_b200 import build as dg_build
+    if rank == 0:
+        dg_build.build()
+    if world > 1:
+        dist.barrier()
+    dg.lib()
+
+    # ---- inputs: one canvas per rank; the embedder is shared model weights
+    E_bits = synth.embedder_normal(V, D, seed=1)
+    h_bits = synth.hidden_normal(B, L, D, seed=2 + 1000 * rank)
+    E = torch.from_numpy(E_bits.view(np.int16)).view(torch.bfloat16).cuda()
+    h = torch.from_numpy(h_bits.view(np.int16)).view(torch.bfloat16).cuda()
+    R = B * L
+    dev = dict(canvas=torch.zeros(R, dtype=torch.int32, device="cuda"),
+               prev=torch.zeros(R, dtype=torch.int32, device="cuda"),
+               acc=torch.zeros(R, dtype=torch.uint8, device="cuda"),
+               ent=torch.zeros(R, dtype=torch.float32, device="cuda"),
+               samp=torch.zeros(R, dtype=torch.int32, device="cuda"),
+               amax=torch.zeros(R, dtype=torch.int32, device="cuda"),
+               stop=torch.zeros(B, dtype=torch.int32, device="cuda"))
+    ws = dg.Workspace(B, D, V)
+    params = dg.Params(seed=1234 + rank)
+    stream = torch.cuda.current_stream()
+
+    def step(i, h_in):
+        dg.denoise_step(h_in, E, [KS[i % 3]], [1 if i > 0 else 0], dev["canvas"], dev["prev"],
+                        dev["acc"], dev["ent"], dev["samp"], dev["amax"], dev["stop"], ws, params)
+
+    def timed_region(K):
+        ev_h = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(K)]
+        for a, b in ev_h:       # torch creates the event handles on first record
+            a.record(stream)
+            b.record(stream)
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for i in range(K):
+            dg.set_head_events(*ev_h[i])
+            step(i, h)
+        dg.set_head_events(None, None)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        total_ms = t0.elapsed_time(t1)
+        head_ms = sum(a.elapsed_time(b) for a, b in ev_h) / K
+        return total_ms, head_ms
+
+    for i in range(args.warmup):
+        step(i, h)
+    torch.cuda.synchronize()
+    assert dg.device_status(ws) == 0
+
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid).replace("GPU-", "")
+    except Exception:
+        gpu_id = str(local)
+    clocks = None
+    for attempt in range(2):
+        sampler = ClockSampler(gpu_id)
+        sampler.start()
+        t_soak = time.time()
+        i = 0
+        while time.time() - t_soak < SOAK_S:      # untimed steady load
+            step(i, h)
+            i += 1
+            if i % 64 == 0:
+                torch.cuda.synchronize()
+        torch.cuda.synchronize()
+        w0 = time.time() - 0.25
+        total_ms, head_ms = timed_region(args.steps)
+        w1 = time.time()
+        rows = sampler.stop()
+        inside = ClockSampler.within(rows, w0, w1)
+        clocks = ClockSampler.summarize(inside if inside else rows)
+        clocks["window"] = ("timed region (+0.25 s of soak before it)" if inside
+                            else "whole sampler run (no timestamped sample in the window)")
+        if not bad_clocks(clocks):
+            break
+        clocks["rejected_first_run"] = True
+    assert dg.device_status(ws) == 0
+
+    # max over ranks
+    t = torch.tensor([total_ms, head_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, head_ms = float(t[0]), float(t[1])
+    ms_per_step = total_ms / args.steps
+    value = world * B * L / (ms_per_step / 1e3)
+
+    # ---- end to end: pinned host h in, results out, through the same API
+    h_host = torch.from_numpy(h_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    h_dev2 = torch.empty_like(h)
+    outs = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory()
+            for k, v in dev.items() if k in ("canvas", "acc", "ent", "stop")}
+    h2d = h_host.numel() * 2
+    d2h = sum(o.numel() * o.element_size() for o in outs.values())
+    K2 = max(1, args.steps)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(K2):
+        h_dev2.copy_(h_host, non_blocking=True)
+        step(i, h_dev2)
+        outs["canvas"].copy_(dev["canvas"], non_blocking=True)
+        outs["acc"].copy_(dev["acc"], non_blocking=True)
+        outs["ent"].copy_(dev["ent"], non_blocking=True)
+        outs["stop"].copy_(dev["stop"], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    et = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(et, op=dist.ReduceOp.MAX)
+        dist.barrier()
+    e2e_ms = float(et[0]) / K2
+    e2e_value = world * B * L / (e2e_ms / 1e3)
+
+    if rank == 0:
+        pk, pk_kind = peaks()
+        alg_bytes = V * D * 2 + R * D * 2
+        achieved = alg_bytes / (head_ms / 1e3) / 1e9
+        traffic, _ = recorded_traffic()
+        flops = 2.0 * R * D * V
+        line = {
+            "metric": METRIC, "value": value, "unit": "slots/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": "B=1 canvas (256 slots) per GPU, d=2816, V=262144, bf16 h and E, "
+                                   "k cycling 0/23/47",
+                       "global_batch": world * B, "seq_len": L, "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (E = 1.48 GB streamed each step)"},
+            "us_per_step": ms_per_step * 1e3,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
+                         "peak_kind": pk_kind, "kernel": "head_sampler_kernel",
+                         "kernel_us": head_ms * 1e3,
+                         "tensor_tflops": flops / (head_ms / 1e3) / 1e12,
+                         "tensor_frac": flops / (head_ms / 1e3) / 1e12 / pk["bf16_tflops"],
+                         "step_roofline_us": max(alg_bytes / (pk["hbm_gbs"] * 1e9),
+                                                 flops / (pk["bf16_tflops"] * 1e12)) * 1e6},
+            "clocks": clocks,
+            "e2e": {"value": e2e_value, "unit": "slots/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": 2 * args.steps,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            t_cpu = oracle_canvas_step(h_bits, E_bits, 0)
+            line["cpu_baseline"] = {"value": L / t_cpu, "unit": "slots/s", "cores": threads_used(),
+                                    "kind": "oracle",
+                                    "sample": "one full B=1 step (256 slots, k=0) of the float64 oracle"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

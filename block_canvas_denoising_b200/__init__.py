@@ -16,7 +16,7 @@ import numpy as np
 
 __all__ = ["DGError", "Params", "lib", "workspace_size", "Workspace", "denoise_step",
            "debug_logits", "device_status", "denoise_loop", "debug_gumbel",
-           "selftest_bounded_wait", "STATUS", "E_BF16", "E_FP8_E4M3"]
+           "selftest_bounded_wait", "set_head_events", "STATUS", "E_BF16", "E_FP8_E4M3"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdg.so")
@@ -92,8 +92,11 @@ def lib() -> ctypes.CDLL:
                                       P, P, P, P, P, P, ctypes.c_size_t, P]
         L.dg_selftest_bounded_wait.argtypes = [ctypes.c_uint64, P, ctypes.c_size_t, P]
         L.dg_debug_gumbel.argtypes = [P, ctypes.c_int32, P, P, P]
+        L.dg_set_head_events.argtypes = [P, P]
+        L.dg_last_error_message.restype = ctypes.c_char_p
         for name in ("dg_workspace_init", "dg_denoise_step", "dg_debug_logits", "dg_device_status",
-                     "dg_denoise_loop", "dg_selftest_bounded_wait", "dg_debug_gumbel"):
+                     "dg_denoise_loop", "dg_selftest_bounded_wait", "dg_debug_gumbel",
+                     "dg_set_head_events"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -101,7 +104,8 @@ def lib() -> ctypes.CDLL:
 
 def _check(code: int, where: str) -> None:
     if code != 0:
-        raise DGError(code, where)
+        msg = lib().dg_last_error_message().decode(errors="replace")
+        raise DGError(code, where + (f" [{msg}]" if msg else ""))
 
 
 def _ptr(t) -> ctypes.c_void_p:
@@ -234,7 +238,8 @@ def denoise_loop(E, hidden_fn, h_buf, canvas, prev_argmax, has_prev, accept, ent
 
 
 def debug_gumbel(words, stream=None):
-    """Device g32 and approximate lg2(E) for uint32 words (torch int32 CUDA tensor)."""
+    """Device g32 and the screening pass's approximate lg2(E / ln 2), E = -ln u,
+    for uint32 words (torch int32 CUDA tensor)."""
     import torch
     n = int(words.numel())
     g = torch.empty(n, dtype=torch.float32, device=words.device)
@@ -242,6 +247,14 @@ def debug_gumbel(words, stream=None):
     _check(lib().dg_debug_gumbel(_ptr(words), ctypes.c_int32(n), _ptr(g), _ptr(a), _stream(stream)),
            "dg_debug_gumbel")
     return g, a
+
+
+def set_head_events(ev_start=None, ev_stop=None) -> None:
+    """Record torch.cuda.Events around the fused head kernel of later steps
+    on this thread (None, None clears)."""
+    a = None if ev_start is None else ctypes.c_void_p(ev_start.cuda_event)
+    b = None if ev_stop is None else ctypes.c_void_p(ev_stop.cuda_event)
+    _check(lib().dg_set_head_events(a, b), "dg_set_head_events")
 
 
 def selftest_bounded_wait(limit_ns: int, ws: Workspace, stream=None) -> int:

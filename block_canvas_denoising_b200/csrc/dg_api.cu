@@ -2,6 +2,7 @@
 // checks, the temperature schedule, TMA descriptors, kernel launches and the
 // adaptive loop.
 #include <cudaTypedefs.h>
+#include <stdio.h>
 #include <string.h>
 
 #include <mutex>
@@ -14,6 +15,19 @@ namespace dg {
 namespace {
 
 constexpr size_t kAlign = 256;
+
+thread_local char t_last_error[256] = "";
+
+// Record a failed CUDA call's message for dg_last_error_message().
+bool cuda_ok(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return true;
+  snprintf(t_last_error, sizeof(t_last_error), "%s: %s (%d)", what, cudaGetErrorString(e),
+           static_cast<int>(e));
+  return false;
+}
+
+thread_local cudaEvent_t t_head_ev_start = nullptr;
+thread_local cudaEvent_t t_head_ev_stop = nullptr;
 size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -125,9 +139,13 @@ dg_status run_step(const StepArgs& a) {
   if (a.logits != nullptr && !aligned16(a.logits)) return DG_ERR_INVALID_ARG;
   for (int b = 0; b < s.B; ++b)
     if (a.step_idx[b] < 0 || a.step_idx[b] >= pr.max_steps) return DG_ERR_RANGE;
-  const int sms = device_sms();
-  if (sms <= 0) return DG_ERR_NO_DEVICE;
-  const WsLayout ws = ws_layout(s, sms);
+  if (device_sms() <= 0) return DG_ERR_NO_DEVICE;
+  const int pairs = head_max_pairs();
+  if (pairs <= 0) {
+    snprintf(t_last_error, sizeof(t_last_error), "no CTA pair of the head kernel fits on this device");
+    return DG_ERR_CUDA;
+  }
+  const WsLayout ws = ws_layout(s, pairs);
   if (a.ws_bytes < ws.total) return DG_ERR_WORKSPACE;
 
   const int R = s.B * s.L;
@@ -142,10 +160,14 @@ dg_status run_step(const StepArgs& a) {
     cps[b].active = (a.active == nullptr || a.active[b]) ? 1 : 0;
   }
 
+  // TMA boxes: one CTA's share of a stage.  The kernel's expect-tx byte
+  // counts and shared-memory slots are sized from the same constants.
+  static_assert(kAStageBytes == kBlockK * kBlockM * 2, "A box / stage mismatch");
+  static_assert(kBStageBytes == kBlockK * kHalfN * 2, "B box / stage mismatch");
   CUtensorMap tmA, tmB;
   if (!encode_2d_bf16(&tmA, a.h, static_cast<uint64_t>(s.d), static_cast<uint64_t>(R), kBlockK, kBlockM))
     return DG_ERR_CUDA;
-  if (!encode_2d_bf16(&tmB, a.E, static_cast<uint64_t>(s.d), static_cast<uint64_t>(s.V), kBlockK, kBlockN))
+  if (!encode_2d_bf16(&tmB, a.E, static_cast<uint64_t>(s.d), static_cast<uint64_t>(s.V), kBlockK, kHalfN))
     return DG_ERR_CUDA;
 
   HeadParams hp;
@@ -154,9 +176,14 @@ dg_status run_step(const StepArgs& a) {
   hp.d = s.d;
   hp.V = s.V;
   hp.B = s.B;
-  hp.split = head_split(R, s.V, s.d, sms);
+  hp.split = head_split(R, s.V, s.d, pairs);
   hp.seed_lo = static_cast<uint32_t>(pr.seed & 0xFFFFFFFFull);
   hp.seed_hi = static_cast<uint32_t>(pr.seed >> 32);
+  // Philox4x32-10 round keys: key + i * (0x9E3779B9, 0xBB67AE85), mod 2^32
+  for (int i = 0; i < 10; ++i) {
+    hp.rk0[i] = hp.seed_lo + static_cast<uint32_t>(i) * 0x9E3779B9u;
+    hp.rk1[i] = hp.seed_hi + static_cast<uint32_t>(i) * 0xBB67AE85u;
+  }
   hp.e_scale = a.e_scale;
   hp.part = reinterpret_cast<float*>(wsb + ws.part_off);
   hp.err = reinterpret_cast<uint32_t*>(wsb + ws.err_off);
@@ -164,7 +191,11 @@ dg_status run_step(const StepArgs& a) {
   hp.wait_ns = kDefaultWaitNs;
   memcpy(hp.cp, cps, sizeof(cps));
 
-  if (launch_head(tmA, tmB, hp, a.stream) != cudaSuccess) return DG_ERR_CUDA;
+  if (t_head_ev_start != nullptr && cudaEventRecord(t_head_ev_start, a.stream) != cudaSuccess)
+    return DG_ERR_CUDA;
+  if (!cuda_ok(launch_head(tmA, tmB, hp, a.stream), "head kernel launch")) return DG_ERR_CUDA;
+  if (t_head_ev_stop != nullptr && cudaEventRecord(t_head_ev_stop, a.stream) != cudaSuccess)
+    return DG_ERR_CUDA;
 
   MergeParams mp;
   memset(&mp, 0, sizeof(mp));
@@ -186,17 +217,17 @@ dg_status run_step(const StepArgs& a) {
   mp.entropy_bound = pr.entropy_bound;
   mp.stop_entropy = pr.stop_entropy;
   memcpy(mp.cp, cps, sizeof(cps));
-  if (launch_merge(mp, a.stream) != cudaSuccess) return DG_ERR_CUDA;
+  if (!cuda_ok(launch_merge(mp, a.stream), "merge kernel launch")) return DG_ERR_CUDA;
   return DG_OK;
 }
 
 }  // namespace
 
-WsLayout ws_layout(const dg_shape& s, int num_sms) {
+WsLayout ws_layout(const dg_shape& s, int max_pairs) {
   WsLayout w;
   const int R = s.B * s.L;
-  const HeadSplit sp = head_split(R, s.V, s.d, num_sms);
-  w.P = 2 * sp.Q;
+  const HeadSplit sp = head_split(R, s.V, s.d, max_pairs);
+  w.P = sp.Q;
   w.err_off = 0;
   w.tickets_off = kAlign;
   w.part_off = align_up(w.tickets_off + sizeof(uint32_t) * static_cast<size_t>(s.B));
@@ -238,9 +269,10 @@ const char* dg_error_string(dg_status s) {
 
 size_t dg_workspace_size(const dg_shape* shape) {
   if (check_shape(shape) != DG_OK) return 0;
-  const int sms = device_sms();
-  if (sms <= 0) return 0;
-  return ws_layout(*shape, sms).total;
+  if (device_sms() <= 0) return 0;
+  const int pairs = head_max_pairs();
+  if (pairs <= 0) return 0;
+  return ws_layout(*shape, pairs).total;
 }
 
 dg_status dg_workspace_init(void* workspace, size_t ws_bytes, void* stream) {
@@ -336,6 +368,15 @@ dg_status dg_denoise_loop(const dg_shape* shape, const dg_params* params, const 
     if (!any) break;
   }
   if (cudaStreamSynchronize(cs) != cudaSuccess) return DG_ERR_CUDA;
+  return DG_OK;
+}
+
+const char* dg_last_error_message(void) { return t_last_error; }
+
+dg_status dg_set_head_events(void* ev_start, void* ev_stop) {
+  if ((ev_start == nullptr) != (ev_stop == nullptr)) return DG_ERR_INVALID_ARG;
+  t_head_ev_start = static_cast<cudaEvent_t>(ev_start);
+  t_head_ev_stop = static_cast<cudaEvent_t>(ev_stop);
   return DG_OK;
 }
 

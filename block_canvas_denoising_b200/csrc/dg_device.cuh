@@ -90,6 +90,46 @@ DG_DEV void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int 
       : "memory");
 }
 
+// Pair variant (tcgen05 cta_group::2): the copy lands in this CTA's shared
+// memory and completes on `bar`, which may be the peer CTA's barrier (a
+// shared::cluster address from mapa).
+DG_DEV void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y,
+                             uint64_t cache_hint) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "l"(cache_hint)
+      : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// clusters
+// ---------------------------------------------------------------------------
+DG_DEV uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+DG_DEV uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+DG_DEV void cluster_sync_all() {
+  asm volatile(
+      "barrier.cluster.arrive.release.aligned;\n\t"
+      "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Arrive on an mbarrier in another CTA of the cluster.
+DG_DEV void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+
 DG_DEV void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -132,6 +172,43 @@ DG_DEV void tc_commit(uint32_t bar) {
                : "memory");
 }
 
+// Pair forms (cta_group::2): TMEM is allocated in both CTAs of the pair by
+// one warp of each; the leader issues the MMA over both CTAs' operands.
+DG_DEV void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+}
+DG_DEV void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+DG_DEV void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+// Arrive once on the barrier at this shared-memory offset in every CTA of
+// `cta_mask` when the pair MMAs issued so far by this thread have completed.
+DG_DEV void tc_commit_pair_mc(uint32_t bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          bar),
+      "h"(cta_mask)
+      : "memory");
+}
+
+// D[tmem of both CTAs] (+)= A[smem of both] * B[smem of both]^T (M = 256 over
+// the pair, N split between the two CTAs' B tiles), bf16, f32 accumulate.
+DG_DEV void tc_mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, f32 accumulate.
 DG_DEV void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                         uint32_t accumulate) {
@@ -165,6 +242,52 @@ DG_DEV uint64_t smem_desc_k_sw128(uint32_t saddr) {
 __host__ __device__ constexpr uint32_t instr_desc_bf16_f32(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Issue a load of 32 consecutive f32 columns of this thread's TMEM lane
+// (32x32b shape).  The registers are valid only after tmem_load_wait(r).
+DG_DEV void tmem_load_issue(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+// Wait for this thread's outstanding TMEM loads; the registers of the last
+// load are tied to the wait so no use is scheduled above it.
+DG_DEV void tmem_load_wait(uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+        "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+        "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),
+        "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
+        "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+      :
+      : "memory");
+}
+
+// Issue a load of 8 consecutive f32 columns of this thread's TMEM lane.
+DG_DEV void tmem_load8_issue(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr)
+               : "memory");
+}
+DG_DEV void tmem_load8_wait(uint32_t (&r)[8]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7])
+               :
+               : "memory");
 }
 
 // 32 consecutive f32 columns of this thread's TMEM lane (32x32b shape), with
@@ -211,6 +334,103 @@ DG_DEV void philox4x32_10(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3, ui
   out[1] = x1;
   out[2] = x2;
   out[3] = x3;
+}
+
+// The ten round keys of a Philox4x32-10 key (k + i * Weyl constants).
+struct PhiloxKeys {
+  uint32_t k0[10], k1[10];
+};
+DG_DEV PhiloxKeys philox_keys(uint32_t k0, uint32_t k1) {
+  PhiloxKeys k;
+#pragma unroll
+  for (int i = 0; i < 10; ++i) {
+    k.k0[i] = k0;
+    k.k1[i] = k1;
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  return k;
+}
+DG_DEV void philox4x32_10_rk(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3, const PhiloxKeys& k,
+                             uint32_t (&out)[4]) {
+#pragma unroll
+  for (int i = 0; i < 10; ++i) {
+    const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * x0;
+    const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * x2;
+    const uint32_t y0 = static_cast<uint32_t>(p1 >> 32) ^ x1 ^ k.k0[i];
+    const uint32_t y2 = static_cast<uint32_t>(p0 >> 32) ^ x3 ^ k.k1[i];
+    x1 = static_cast<uint32_t>(p1);
+    x3 = static_cast<uint32_t>(p0);
+    x0 = y0;
+    x2 = y2;
+  }
+  out[0] = x0;
+  out[1] = x1;
+  out[2] = x2;
+  out[3] = x3;
+}
+
+// Same, with the round keys in two arrays (e.g. kernel parameters).
+DG_DEV void philox4x32_10_keys(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3,
+                               const uint32_t (&k0)[10], const uint32_t (&k1)[10], uint32_t (&out)[4]) {
+#pragma unroll
+  for (int i = 0; i < 10; ++i) {
+    const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * x0;
+    const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * x2;
+    const uint32_t y0 = static_cast<uint32_t>(p1 >> 32) ^ x1 ^ k0[i];
+    const uint32_t y2 = static_cast<uint32_t>(p0 >> 32) ^ x3 ^ k1[i];
+    x1 = static_cast<uint32_t>(p1);
+    x3 = static_cast<uint32_t>(p0);
+    x0 = y0;
+    x2 = y2;
+  }
+  out[0] = x0;
+  out[1] = x1;
+  out[2] = x2;
+  out[3] = x3;
+}
+
+// ---------------------------------------------------------------------------
+// Per-row partial of the fused head: base-2 online softmax of x = z / tau
+// (m2 = max x log2 e, S = sum 2^(x log2 e - m2), T2 = sum (x log2 e - m2)
+// 2^(...)), argmax of z, best specified Gumbel key.
+// ---------------------------------------------------------------------------
+struct Partial {
+  float m2, S, T2;
+  float zmax;
+  int zarg;
+  float gkey;
+  int garg;
+};
+
+DG_DEV void partial_init(Partial& a) {
+  a.m2 = -1.0e30f;
+  a.S = 0.f;
+  a.T2 = 0.f;
+  a.zmax = -3.402823466e38f;
+  a.zarg = 0x7fffffff;
+  a.gkey = -3.402823466e38f;
+  a.garg = 0x7fffffff;
+}
+
+// Merge b into a.  Softmax: m = max(m_a, m_b), S = sum_i S_i 2^(m_i - m),
+// T2 = sum_i (T2_i + (m_i - m) S_i) 2^(m_i - m).  Argmax and Gumbel key: the
+// larger value wins, ties to the lower vocabulary index.
+DG_DEV void partial_merge(Partial& a, const Partial& b) {
+  const float m = fmaxf(a.m2, b.m2);
+  const float da = a.m2 - m, db = b.m2 - m;
+  const float sa = exp2f(da), sb = exp2f(db);
+  a.T2 = (a.T2 + da * a.S) * sa + (b.T2 + db * b.S) * sb;
+  a.S = a.S * sa + b.S * sb;
+  a.m2 = m;
+  if (b.zmax > a.zmax || (b.zmax == a.zmax && b.zarg < a.zarg)) {
+    a.zmax = b.zmax;
+    a.zarg = b.zarg;
+  }
+  if (b.gkey > a.gkey || (b.gkey == a.gkey && b.garg < a.garg)) {
+    a.gkey = b.gkey;
+    a.garg = b.garg;
+  }
 }
 
 // Stream purposes (high half of counter word 1).
@@ -286,24 +506,30 @@ DG_DEV float ex2_approx(float x) {
   return y;
 }
 
-// log2 of the Exp(1) variable E = -ln u, approximately.  For u > 15/16
-// (y = 1 - u < 1/16, where lg2 of u loses relative accuracy) E comes from
-// -ln(1 - y) = y (1 + y/2 + y^2/3 + y^3/4 + ...); otherwise from the fast
-// hardware log2.  Returns lg2(E) so that g = -ln 2 * lg2(E).  The result's
-// distance from the exact transform is measured over all 2^23 inputs by the
-// GPU tests and bounded by kGumbelApproxErr.
+// Screening transform.  With E = -ln u (an Exp(1) variable) and
+// E2 = E / ln 2 = -lg2 u, the Gumbel noise is g = -ln E = C0 - ln2 lg2(E2)
+// with C0 = -ln(ln 2).  This returns an approximation of lg2(E2): for
+// u > 15/16 (y = 1 - u < 1/16, where the hardware lg2 of u loses relative
+// accuracy) E2 comes from -lg2(1 - y) = (y + y^2/2 + y^3/3 + y^4/4 + ...)/ln 2,
+// otherwise from the hardware lg2.  Its distance from the specified g32 is
+// measured over all 2^23 inputs by the GPU tests and bounded by
+// kGumbelApproxErr.
 DG_DEV float lg2_exp1_approx(uint32_t r) {
   const float one_plus = __uint_as_float((r >> 9) | 0x3F800000u);  // 1 + r23 2^-23
   const float u = __fsub_rn(one_plus, __uint_as_float(0x3f7fffffu));  // - (1 - 2^-24), exact
   const float y = __fsub_rn(1.0f, u);                                 // exact
-  float t = __fmaf_rn(y, 0.25f, __uint_as_float(0x3eaaaaabu));        // 1/3 + y/4
-  t = __fmaf_rn(y, t, 0.5f);
-  t = __fmaf_rn(y, t, 1.0f);
-  const float e_series = __fmul_rn(y, t);
-  const float e_log = __fmul_rn(lg2_approx(u), -0.693147182464599609375f);
-  const float e = (y < 0.0625f) ? e_series : e_log;
-  return lg2_approx(e);
+  // -(y/ln2)(1 + y/2 + y^2/3 + y^3/4): coefficients -1/(k ln 2)
+  float t = __fmaf_rn(y, -0.36067376022224085f, -0.48089834696298783f);
+  t = __fmaf_rn(y, t, -0.72134752044448170f);
+  t = __fmaf_rn(y, t, -1.44269504088896341f);
+  const float neg_e2_series = __fmul_rn(y, t);
+  const float neg_e2_log = lg2_approx(u);  // lg2 u = -E2
+  const float neg_e2 = (y < 0.0625f) ? neg_e2_series : neg_e2_log;
+  return lg2_approx(-neg_e2);
 }
+
+// C0 = -ln(ln 2): g = C0 - ln2 * lg2(E2).
+constexpr float kGumbelC0 = 0.36651292058166432f;
 
 // |approx key - specified key| <= kGumbelApproxErr + rounding of the keys.
 constexpr float kGumbelApproxErr = 1.0e-5f;

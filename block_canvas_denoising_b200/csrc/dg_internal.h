@@ -10,18 +10,27 @@
 
 namespace dg {
 
-// Tile of the fused head+sampler kernel: 128 canvas rows x 256 vocabulary
-// columns, K staged 64 bf16 (128 B, one swizzle row) at a time.
-constexpr int kBlockM = 128;
-constexpr int kBlockN = 256;
+// Tile of the fused head+sampler kernel.  A CTA pair (cluster of 2, tcgen05
+// cta_group::2) computes 256 canvas rows x 256 vocabulary columns per tile;
+// each CTA stages 128 rows of h and 128 rows of E per 64-wide K block (one
+// 128-byte swizzle row) and holds its 128 x 256 float32 half in TMEM.
+constexpr int kPairM = 256;                       // rows per pair tile
+constexpr int kBlockM = 128;                      // rows per CTA
+constexpr int kBlockN = 256;                      // vocabulary columns per tile
+constexpr int kHalfN = 128;                       // E rows staged per CTA
 constexpr int kBlockK = 64;
-constexpr int kStages = 4;
-constexpr int kEpiWarps = 8;                      // 2 column groups x 4 lane quarters
-constexpr int kHeadThreads = 64 + kEpiWarps * 32; // producer, MMA, epilogue
+constexpr int kStages = 6;
+constexpr int kEpiWarps = 16;                     // 4 column groups x 4 lane quarters
+constexpr int kColGroups = kEpiWarps / 4;         // 64 columns each
+constexpr int kProducerWarp = kEpiWarps;          // warp 16
+constexpr int kMmaWarp = kEpiWarps + 1;           // warp 17
+constexpr int kHeadThreads = (kEpiWarps + 2) * 32;
 constexpr int kAStageBytes = kBlockM * kBlockK * 2;
-constexpr int kBStageBytes = kBlockN * kBlockK * 2;
-constexpr int kHeadSmemBytes = kStages * (kAStageBytes + kBStageBytes) + 1024 + 256;
+constexpr int kBStageBytes = kHalfN * kBlockK * 2;
 constexpr int kPartialFields = 7;                 // m2, S, T2, zmax, zarg, gkey, garg
+// per-unit exchange of the column groups' partials inside a CTA
+constexpr int kPartSmemBytes = kColGroups * kBlockM * kPartialFields * 4;
+constexpr int kHeadSmemBytes = kStages * (kAStageBytes + kBStageBytes) + 1024 + 256 + kPartSmemBytes;
 constexpr uint64_t kDefaultWaitNs = 4000000000ull;
 
 // Per-canvas step data, filled on the host.
@@ -33,11 +42,12 @@ struct CanvasParam {
   uint8_t pad[2];
 };
 
-// Work split of the head: MT row tiles x NT vocabulary tiles, cut into
-// units of consecutive vocabulary tiles of one row tile.  Unit u covers row
-// tile u % MT and vocabulary tiles [q NT / Q, (q+1) NT / Q), q = u / MT.
+// Work split of the head: MT pair row tiles (256 rows) x NT vocabulary
+// tiles, cut into units of consecutive vocabulary tiles of one row tile.
+// Unit u covers row tile u % MT and vocabulary tiles [q NT / Q, (q+1) NT / Q),
+// q = u / MT; pair p runs units p, p + pairs, ...  grid = 2 * pairs CTAs.
 struct HeadSplit {
-  int MT, NT, KB, Q, units, grid;
+  int MT, NT, KB, Q, units, pairs, grid;
 };
 
 struct HeadParams {
@@ -45,10 +55,11 @@ struct HeadParams {
   HeadSplit split;
   uint32_t seed_lo, seed_hi;
   const float* e_scale;  // per-vocabulary-row scale (FP8) or null
-  float* part;           // partial records, kPartialFields planes of [2Q][R]
+  float* part;           // partial records, kPartialFields planes of [R][Q]
   uint32_t* err;         // device fault latch
   float* logits_out;     // optional raw logits [R, V]
   uint64_t wait_ns;
+  uint32_t rk0[10], rk1[10];  // Philox round keys of the seed
   CanvasParam cp[DG_MAX_B];
 };
 
@@ -69,14 +80,15 @@ struct MergeParams {
   CanvasParam cp[DG_MAX_B];
 };
 
-HeadSplit head_split(int R, int V, int d, int num_sms);
+HeadSplit head_split(int R, int V, int d, int max_pairs);
+int head_max_pairs();
 
 // Workspace layout (byte offsets), see dg_workspace_size().
 struct WsLayout {
   size_t err_off, tickets_off, part_off, total;
   int P;
 };
-WsLayout ws_layout(const dg_shape& s, int num_sms);
+WsLayout ws_layout(const dg_shape& s, int max_pairs);
 
 cudaError_t launch_head(const CUtensorMap& tmA, const CUtensorMap& tmB, const HeadParams& p,
                         cudaStream_t stream);

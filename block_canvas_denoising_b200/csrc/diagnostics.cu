@@ -3,7 +3,7 @@
 //     nobody arrives at and must give up after `limit_ns`, latching
 //     kErrSelftest, with the context left usable;
 //   * a probe of the Gumbel transforms on given Philox words: the specified
-//     IEEE-only g32 and the approximate lg2(E) the screening pass uses.
+//     IEEE-only g32 and the approximate lg2(E / ln 2) the screening pass uses.
 #include "dg_device.cuh"
 #include "dg_internal.h"
 

@@ -14,9 +14,15 @@
 //   * the Gumbel-max draw argmax_v fl(fl(z_v / tau) + g32(u_v)) with u_v
 //     from Philox4x32-10 counter (v >> 2, slot, k, b), lane v & 3.
 //
-// Warp roles (320 threads, one CTA per SM, persistent):
-//   warp 0      TMA producer: h and E tiles -> 4-stage shared-memory ring.
-//   warp 1      TMEM allocator and MMA issuer (tcgen05.mma, 128x256x16 bf16).
+// The kernel runs as CTA pairs (clusters of 2) on the tcgen05 cta_group::2
+// path: the pair computes 256 rows x 256 vocabulary columns per tile, the
+// leader CTA issuing 256x256x16 bf16 MMAs over both CTAs' shared memory;
+// each CTA holds its 128-row half of the tile in its own TMEM.
+//
+// Warp roles (320 threads per CTA, one CTA per SM, persistent):
+//   warp 0      TMA producer: this CTA's halves of the h and E tiles into a
+//               6-stage shared-memory ring (completion on the leader's barrier).
+//   warp 1      TMEM allocator; in the leader, the MMA issuer.
 //   warps 2..9  epilogue: warp w reads TMEM lane quarter w % 4 and column
 //               half (w - 2) / 4 of each tile; two accumulators alternate
 //               so the epilogue of tile t overlaps the MMAs of tile t + 1.
@@ -29,14 +35,6 @@
 namespace dg {
 
 namespace {
-
-struct Partial {
-  float m2, S, T2;  // base-2 online softmax of x = z * inv_tau
-  float zmax;       // argmax of z
-  int zarg;
-  float gkey;       // best specified Gumbel key so far
-  int garg;
-};
 
 DG_DEV void unit_range(const HeadSplit& sp, int u, int& m, int& n0, int& n1, int& q) {
   q = u / sp.MT;
@@ -54,35 +52,82 @@ DG_DEV void gumbel_update(Partial& pt, float key, int v) {
   }
 }
 
-// One 32-column chunk of one row: z[0..31] are logits v0 .. v0+31.
-DG_DEV void process_chunk(const float (&z)[32], int v0, float inv_tau, float c2, uint32_t ctr1,
-                          uint32_t ctr2, uint32_t ctr3, uint32_t k0, uint32_t k1, Partial& pt) {
-  // ---- argmax of z (ties to the lower index; chunks arrive in increasing v)
-  float cmax = z[0];
+// The specified key of one element, kept out of line: it is needed rarely,
+// and inlining it at every call site would bloat the epilogue's loop.
+__device__ __noinline__ float key_exact_call(float z, float inv_tau, uint32_t w) {
+  return key_exact(z, inv_tau, w);
+}
+
+DG_DEV void confirm_exact(Partial& pt, float z, float inv_tau, uint32_t w, int v) {
+  gumbel_update(pt, key_exact_call(z, inv_tau, w), v);
+}
+
+// Streaming state of the Gumbel screen.  Every element gets a screening key
+// ka within e of its specified key (kGumbelApproxErr plus roundings); keys
+// are packed with the element's index in their 3 lowest bits, which moves
+// them by at most 7 ulps.  Per group of 8 the largest two packed keys
+// (K1g, K2g) are found branch-free; with eps above twice the combined error:
+//   * K1g < K1a - eps: nothing in the group can beat the pending candidate;
+//   * a near-tie (K2g >= K1g - eps inside the group, or |K1g - K1a| <= eps)
+//     confirms exactly every group element within eps of K1g (rare);
+//   * K1g > K1a + eps: the group's best becomes the pending candidate (the
+//     old one is then certainly worse).
+// The pending candidate is confirmed exactly at the end of each unit.
+struct Screen {
+  float K1a;       // packed screening key of the pending candidate (-inf if none)
+  float z1;        // its logit
+  uint32_t w1;     // its Philox word
+  int v1;          // its vocabulary index
+};
+
+DG_DEV float screen_eps(float k) {
+  return 2.0f * kGumbelApproxErr + (fabsf(k) + 64.0f) * 1.9073486328125e-06f;  // 2^-19
+}
+
+DG_DEV void screen_reset(Screen& sc) { sc.K1a = -FLT_MAX; }
+
+DG_DEV void screen_flush(Screen& sc, Partial& pt, float inv_tau) {
+  if (sc.K1a > -FLT_MAX) confirm_exact(pt, sc.z1, inv_tau, sc.w1, sc.v1);
+  screen_reset(sc);
+}
+
+DG_DEV void top2(float& a1, float& a2, float b1, float b2) {
+  const float hi = fmaxf(a1, b1);
+  a2 = fmaxf(fminf(a1, b1), fmaxf(a2, b2));
+  a1 = hi;
+}
+
+// Eight consecutive logits of one row: z[0..7] are vocabulary v0 .. v0+7.
+DG_DEV void process8(const float (&z)[8], int v0, float inv_tau, float c2, uint32_t ctr1,
+                     uint32_t ctr2, uint32_t ctr3, const uint32_t (&rk0)[10], const uint32_t (&rk1)[10],
+                     Partial& pt, Screen& sc) {
+  // ---- group max, argmax of z (ties to the lower index; groups arrive in
+  // increasing v)
+  const float m01 = fmaxf(z[0], z[1]), m23 = fmaxf(z[2], z[3]);
+  const float m45 = fmaxf(z[4], z[5]), m67 = fmaxf(z[6], z[7]);
+  const float gmax = fmaxf(fmaxf(m01, m23), fmaxf(m45, m67));
+  if (gmax > pt.zmax) {
+    int jj = 7;
 #pragma unroll
-  for (int j = 1; j < 32; ++j) cmax = fmaxf(cmax, z[j]);
-  if (cmax > pt.zmax) {
-    int jj = 0;
-#pragma unroll
-    for (int j = 31; j >= 0; --j) jj = (z[j] == cmax) ? j : jj;
-    pt.zmax = cmax;
+    for (int j = 6; j >= 0; --j) jj = (z[j] == gmax) ? j : jj;
+    pt.zmax = gmax;
     pt.zarg = v0 + jj;
   }
 
   // ---- online softmax partial, base 2
-  const float cm2 = cmax * c2;
-  if (cm2 > pt.m2) {
-    const float delta = pt.m2 - cm2;
-    const float sc = ex2_approx(delta);
-    pt.T2 = (pt.T2 + delta * pt.S) * sc;
-    pt.S = pt.S * sc;
-    pt.m2 = cm2;
+  const float gm2 = gmax * c2;
+  if (gm2 > pt.m2) {
+    const float delta = pt.m2 - gm2;
+    const float scl = ex2_approx(delta);
+    pt.T2 = (pt.T2 + delta * pt.S) * scl;
+    pt.S = pt.S * scl;
+    pt.m2 = gm2;
   }
   {
-    float s0 = 0.f, s1 = 0.f, t0 = 0.f, t1 = 0.f;
     const float nm = -pt.m2;
+    float s0 = 0.f, s1 = 0.f, t0 = 0.f, t1 = 0.f;
 #pragma unroll
-    for (int j = 0; j < 32; j += 2) {
+    for (int j = 0; j < 8; j += 2) {
       const float d0 = fmaf(z[j], c2, nm);
       const float d1 = fmaf(z[j + 1], c2, nm);
       const float e0 = ex2_approx(d0);
@@ -96,53 +141,91 @@ DG_DEV void process_chunk(const float (&z)[32], int v0, float inv_tau, float c2,
     pt.T2 += t0 + t1;
   }
 
-  // ---- Gumbel-max: screen with the approximate key, confirm exactly
-  const uint32_t cbase = static_cast<uint32_t>(v0) >> 2;
-  float K1 = -FLT_MAX, K2 = -FLT_MAX, zK1 = 0.f;
-  int j1 = 0;
-#pragma unroll
-  for (int q4 = 0; q4 < 8; ++q4) {
-    uint32_t r[4];
-    philox4x32_10(cbase + q4, ctr1, ctr2, ctr3, k0, k1, r);
+  // ---- Gumbel-max screen (branch-free except for rare near-ties)
+  const uint32_t cb = static_cast<uint32_t>(v0) >> 2;
+  uint32_t w[8];
+  {
+    uint32_t wa[4], wb[4];
+    philox4x32_10_keys(cb, ctr1, ctr2, ctr3, rk0, rk1, wa);
+    philox4x32_10_keys(cb + 1, ctr1, ctr2, ctr3, rk0, rk1, wb);
 #pragma unroll
     for (int l = 0; l < 4; ++l) {
-      const int j = 4 * q4 + l;
-      const float x = __fmul_rn(z[j], inv_tau);
-      const float ka = __fmaf_rn(lg2_exp1_approx(r[l]), -kLn2, x);
-      const bool p = ka > K1;
-      K2 = fmaxf(K2, p ? K1 : ka);
-      zK1 = p ? z[j] : zK1;
-      j1 = p ? j : j1;
-      K1 = p ? ka : K1;
+      w[l] = wa[l];
+      w[4 + l] = wb[l];
     }
   }
-  // Any specified key differs from its approximate key by at most
-  // kGumbelApproxErr plus the roundings of the two keys; eps is twice that
-  // bound with room to spare.
-  const float eps = 2.0f * kGumbelApproxErr + (fabsf(K1) + 64.0f) * 9.5367431640625e-07f;
-  if (K1 >= pt.gkey - eps) {
-    if (K2 >= K1 - eps) {
-      // near-tie inside the chunk: confirm every element
+  float kp[8];
 #pragma unroll
-      for (int q4 = 0; q4 < 8; ++q4) {
-        uint32_t r[4];
-        philox4x32_10(cbase + q4, ctr1, ctr2, ctr3, k0, k1, r);
-#pragma unroll
-        for (int l = 0; l < 4; ++l) gumbel_update(pt, key_exact(z[4 * q4 + l], inv_tau, r[l]), v0 + 4 * q4 + l);
-      }
-    } else {
-      uint32_t r[4];
-      philox4x32_10(cbase + (static_cast<uint32_t>(j1) >> 2), ctr1, ctr2, ctr3, k0, k1, r);
-      const int l = j1 & 3;
-      const uint32_t rw = (l == 0) ? r[0] : (l == 1) ? r[1] : (l == 2) ? r[2] : r[3];
-      gumbel_update(pt, key_exact(zK1, inv_tau, rw), v0 + j1);
-    }
+  for (int j = 0; j < 8; ++j) {
+    const float x0 = __fmaf_rn(z[j], inv_tau, kGumbelC0);
+    const float ka = __fmaf_rn(lg2_exp1_approx(w[j]), -kLn2, x0);
+    kp[j] = __int_as_float((__float_as_int(ka) & ~7) | j);
   }
+  float a1 = fmaxf(kp[0], kp[1]), a2 = fminf(kp[0], kp[1]);
+  float b1 = fmaxf(kp[2], kp[3]), b2 = fminf(kp[2], kp[3]);
+  float c1 = fmaxf(kp[4], kp[5]), c2b = fminf(kp[4], kp[5]);
+  float d1 = fmaxf(kp[6], kp[7]), d2 = fminf(kp[6], kp[7]);
+  top2(a1, a2, b1, b2);
+  top2(c1, c2b, d1, d2);
+  top2(a1, a2, c1, c2b);
+  const float K1g = a1, K2g = a2;
+  const float eps = screen_eps(K1g);
+  if (K1g >= sc.K1a - eps && (K2g >= K1g - eps || K1g <= sc.K1a + eps)) {
+    const float lo = K1g - eps;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (kp[j] >= lo) confirm_exact(pt, z[j], inv_tau, w[j], v0 + j);
+  }
+  if (K1g > sc.K1a + eps) {
+    const int j1 = __float_as_int(K1g) & 7;
+    float zs = z[0];
+    uint32_t ws = w[0];
+#pragma unroll
+    for (int j = 1; j < 8; ++j) {
+      zs = (j == j1) ? z[j] : zs;
+      ws = (j == j1) ? w[j] : ws;
+    }
+    sc.K1a = K1g;
+    sc.z1 = zs;
+    sc.w1 = ws;
+    sc.v1 = v0 + j1;
+  }
+}
+
+// Scale (FP8 embedder), optional logits dump, then the group's reductions.
+DG_DEV void epi_group(const uint32_t (&r)[8], int v0, int row, float inv_tau, float c2, uint32_t ctr1,
+                      uint32_t ctr2, uint32_t ctr3, const HeadParams& p, Partial& pt, Screen& sc) {
+  float z[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) z[j] = __uint_as_float(r[j]);
+  if (p.e_scale != nullptr) {
+    const float4* scp = reinterpret_cast<const float4*>(p.e_scale + v0);
+    const float4 s0 = __ldg(scp), s1 = __ldg(scp + 1);
+    z[0] = __fmul_rn(z[0], s0.x);
+    z[1] = __fmul_rn(z[1], s0.y);
+    z[2] = __fmul_rn(z[2], s0.z);
+    z[3] = __fmul_rn(z[3], s0.w);
+    z[4] = __fmul_rn(z[4], s1.x);
+    z[5] = __fmul_rn(z[5], s1.y);
+    z[6] = __fmul_rn(z[6], s1.z);
+    z[7] = __fmul_rn(z[7], s1.w);
+  }
+  if (p.logits_out != nullptr) {
+    float4* dst = reinterpret_cast<float4*>(p.logits_out + static_cast<size_t>(row) * p.V + v0);
+    dst[0] = make_float4(z[0], z[1], z[2], z[3]);
+    dst[1] = make_float4(z[4], z[5], z[6], z[7]);
+  }
+  process8(z, v0, inv_tau, c2, ctr1, ctr2, ctr3, p.rk0, p.rk1, pt, sc);
+}
+
+// Named barrier over the epilogue warps only (barrier 1).
+DG_DEV void epilogue_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
 }
 
 }  // namespace
 
-__global__ void __launch_bounds__(kHeadThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kHeadThreads, 1)
 head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ HeadParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -151,9 +234,15 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   uint8_t* sB = smem + kStages * kAStageBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sB + kStages * kBStageBytes);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 4);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // [column group][field][row of the CTA half]
+  float* sPart = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0 = leader (issues the MMAs), 1 = peer
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
   const HeadSplit& sp = p.split;
 
   auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
@@ -165,33 +254,37 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1);
+      mbar_init(full_bar(s), 1);   // leader's producer arrival + both CTAs' bytes
+      mbar_init(empty_bar(s), 1);  // one multicast commit per use
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), kEpiWarps);
+      mbar_init(tfull_bar(a), 1);               // one multicast commit per tile
+      mbar_init(tempty_bar(a), 2 * kEpiWarps);  // every epilogue warp of the pair
     }
+    *s_abort = 0;
     fence_mbarrier_init();
   }
-  if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), 2 * kBlockN);
-    tmem_relinquish();
+  if (warp == kMmaWarp) {
+    tmem_alloc_pair(smem_u32(tmem_slot), 2 * kBlockN);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
+    // Each CTA loads its own halves: 128 rows of h (rows rank*128 of the
+    // pair tile) and 128 rows of E (the rank-th half of the 256 vocabulary
+    // columns).  All copies complete on the leader's full barrier.
     if (lane == 0) {
-      const uint64_t pol_h = policy_evict_last();   // h is re-read by every unit
+      const uint64_t pol_h = policy_evict_last();   // h is re-read by every tile
       const uint64_t pol_e = policy_evict_first();  // E streams through once
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < sp.units && ok; u += gridDim.x) {
+      for (int u = pair; u < sp.units && ok; u += npairs) {
         int m, n0, n1, q;
         unit_range(sp, u, m, n0, n1, q);
         for (int n = n0; n < n1 && ok; ++n) {
@@ -201,11 +294,13 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
               ok = false;
               break;
             }
-            mbar_arrive_expect_tx(full_bar(stage), kAStageBytes + kBStageBytes);
-            tma_load_2d(smem_u32(sA + stage * kAStageBytes), &tmA, full_bar(stage), kb * kBlockK,
-                        m * kBlockM, pol_h);
-            tma_load_2d(smem_u32(sB + stage * kBStageBytes), &tmB, full_bar(stage), kb * kBlockK,
-                        n * kBlockN, pol_e);
+            const uint32_t fb = full_bar(stage);
+            if (rank == 0) mbar_arrive_expect_tx(fb, 2 * (kAStageBytes + kBStageBytes));
+            const uint32_t fb_leader = mapa_shared(fb, 0);
+            tma_load_2d_pair(smem_u32(sA + stage * kAStageBytes), &tmA, fb_leader, kb * kBlockK,
+                             m * kPairM + static_cast<int>(rank) * kBlockM, pol_h);
+            tma_load_2d_pair(smem_u32(sB + stage * kBStageBytes), &tmB, fb_leader, kb * kBlockK,
+                             n * kBlockN + static_cast<int>(rank) * kHalfN, pol_e);
             if (++stage == kStages) {
               stage = 0;
               phase ^= 1u;
@@ -213,16 +308,28 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           }
         }
       }
+      // Tail: wait until the MMAs have released every stage, so no commit
+      // arrival can land in this CTA's shared memory after it exits.
+      for (int i = 0; i < kStages && ok; ++i) {
+        if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, p.wait_ns)) {
+          latch_error(p.err, kErrWaitTmaProducer);
+          ok = false;
+        }
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = instr_desc_bf16_f32(kBlockM, kBlockN);
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = instr_desc_bf16_f32(kPairM, kBlockN);
       int stage = 0;
       uint32_t phase = 0;
       int tile = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < sp.units && ok; u += gridDim.x) {
+      for (int u = pair; u < sp.units && ok; u += npairs) {
         int m, n0, n1, q;
         unit_range(sp, u, m, n0, n1, q);
         for (int n = n0; n < n1 && ok; ++n, ++tile) {
@@ -247,32 +354,32 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 #pragma unroll
             for (int k16 = 0; k16 < kBlockK / 16; ++k16) {
               // advance 16 bf16 = 32 B along K inside the swizzled rows
-              tc_mma_bf16(d_tmem, adesc + 2u * k16, bdesc + 2u * k16, idesc,
-                          (kb > 0 || k16 > 0) ? 1u : 0u);
+              tc_mma_bf16_pair(d_tmem, adesc + 2u * k16, bdesc + 2u * k16, idesc,
+                               (kb > 0 || k16 > 0) ? 1u : 0u);
             }
-            tc_commit(empty_bar(stage));
+            tc_commit_pair_mc(empty_bar(stage), 0x3);  // frees the stage in both CTAs
             if (++stage == kStages) {
               stage = 0;
               phase ^= 1u;
             }
           }
-          if (ok) tc_commit(tfull_bar(acc));
+          if (ok) tc_commit_pair_mc(tfull_bar(acc), 0x3);
         }
       }
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int ew = warp - 2;
     const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
-    const int cg = ew >> 2;        // column half of the tile
-    const uint32_t k0 = p.seed_lo, k1 = p.seed_hi;
-    const int P = 2 * sp.Q;
+    const int cg = warp >> 2;      // 64-column group of the tile
+    const int rloc = quarter * 32 + lane;
+    // Every epilogue warp runs the same units and named barriers even after
+    // a failed wait (it then skips the work), so the barriers cannot deadlock.
     int tile = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < sp.units && ok; u += gridDim.x) {
+    for (int u = pair; u < sp.units; u += npairs) {
       int m, n0, n1, q;
       unit_range(sp, u, m, n0, n1, q);
-      const int row = m * kBlockM + quarter * 32 + lane;
+      const int row = m * kPairM + static_cast<int>(rank) * kBlockM + rloc;
       const int b = row >> 8;
       const int slot = row & 255;
       const CanvasParam cp = p.cp[b];
@@ -282,105 +389,150 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       const uint32_t ctr2 = static_cast<uint32_t>(cp.k);
       const uint32_t ctr3 = static_cast<uint32_t>(b);
       Partial pt;
-      pt.m2 = -1.0e30f;
-      pt.S = 0.f;
-      pt.T2 = 0.f;
-      pt.zmax = -FLT_MAX;
-      pt.zarg = INT_MAX;
-      pt.gkey = -FLT_MAX;
-      pt.garg = INT_MAX;
+      partial_init(pt);
+      Screen sc;
+      screen_reset(sc);
       for (int n = n0; n < n1; ++n, ++tile) {
         const int acc = tile & 1;
         const uint32_t acc_phase = (tile >> 1) & 1;
+        if (ok && *s_abort) ok = false;
+        if (!ok) continue;
         if (!mbar_wait_bounded(tfull_bar(acc), acc_phase, p.wait_ns)) {
           latch_error(p.err, kErrWaitEpilogue);
+          *s_abort = 1;
           ok = false;
-          break;
+          continue;
         }
         tc_fence_after();
+        // 8 groups of 8 columns; the TMEM load of group g+1 is in flight
+        // while group g is processed
+        constexpr int kGroups = kBlockN / kColGroups / 8;
+        const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                               static_cast<uint32_t>(acc * kBlockN + cg * (kBlockN / kColGroups));
+        const int vbase = n * kBlockN + cg * (kBlockN / kColGroups);
+        uint32_t ra[8], rb[8];
+        __syncwarp();
+        tmem_load8_issue(tbase, ra);
+        tmem_load8_wait(ra);
 #pragma unroll 1
-        for (int c = 0; c < kBlockN / 2 / 32; ++c) {
-          const int col = acc * kBlockN + cg * (kBlockN / 2) + c * 32;
-          const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + col;
-          float z[32];
+        for (int g = 0; g < kGroups; g += 2) {
+          tmem_load8_issue(tbase + 8 * (g + 1), rb);
+          epi_group(ra, vbase + 8 * g, row, inv_tau, c2, ctr1, ctr2, ctr3, p, pt, sc);
+          tmem_load8_wait(rb);
+          if (g + 2 < kGroups) tmem_load8_issue(tbase + 8 * (g + 2), ra);
+          epi_group(rb, vbase + 8 * (g + 1), row, inv_tau, c2, ctr1, ctr2, ctr3, p, pt, sc);
+          tmem_load8_wait(ra);
           __syncwarp();
-          tmem_load_32cols(taddr, z);
-          const int v0 = n * kBlockN + cg * (kBlockN / 2) + c * 32;
-          if (p.e_scale != nullptr) {
-            const float4* sc = reinterpret_cast<const float4*>(p.e_scale + v0);
-#pragma unroll
-            for (int j4 = 0; j4 < 8; ++j4) {
-              const float4 s4 = __ldg(sc + j4);
-              z[4 * j4 + 0] = __fmul_rn(z[4 * j4 + 0], s4.x);
-              z[4 * j4 + 1] = __fmul_rn(z[4 * j4 + 1], s4.y);
-              z[4 * j4 + 2] = __fmul_rn(z[4 * j4 + 2], s4.z);
-              z[4 * j4 + 3] = __fmul_rn(z[4 * j4 + 3], s4.w);
-            }
-          }
-          if (p.logits_out != nullptr) {
-            float4* dst = reinterpret_cast<float4*>(p.logits_out + static_cast<size_t>(row) * p.V + v0);
-#pragma unroll
-            for (int j4 = 0; j4 < 8; ++j4)
-              dst[j4] = make_float4(z[4 * j4], z[4 * j4 + 1], z[4 * j4 + 2], z[4 * j4 + 3]);
-          }
-          process_chunk(z, v0, inv_tau, c2, ctr1, ctr2, ctr3, k0, k1, pt);
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(tempty_bar(acc));
+        if (lane == 0) {
+          if (rank == 0)
+            mbar_arrive(tempty_bar(acc));
+          else
+            mbar_arrive_remote(mapa_shared(tempty_bar(acc), 0));
+        }
       }
-      if (!ok) break;
-      // one partial record per (row, unit, column half), planes of [P][R]
-      const size_t plane = static_cast<size_t>(P) * p.R;
-      const size_t idx = static_cast<size_t>(2 * q + cg) * p.R + row;
-      float* part = p.part;
-      part[0 * plane + idx] = pt.m2;
-      part[1 * plane + idx] = pt.S;
-      part[2 * plane + idx] = pt.T2;
-      part[3 * plane + idx] = pt.zmax;
-      part[4 * plane + idx] = __int_as_float(pt.zarg);
-      part[5 * plane + idx] = pt.gkey;
-      part[6 * plane + idx] = __int_as_float(pt.garg);
+      if (ok) screen_flush(sc, pt, inv_tau);
+      // ---- merge the column groups' partials of each row in the CTA, then
+      // write one record per (row, unit): planes of [R][Q]
+      if (cg != 0) {
+        float* d = sPart + (cg * kPartialFields) * kBlockM + rloc;
+        d[0 * kBlockM] = pt.m2;
+        d[1 * kBlockM] = pt.S;
+        d[2 * kBlockM] = pt.T2;
+        d[3 * kBlockM] = pt.zmax;
+        d[4 * kBlockM] = __int_as_float(pt.zarg);
+        d[5 * kBlockM] = pt.gkey;
+        d[6 * kBlockM] = __int_as_float(pt.garg);
+      }
+      epilogue_sync();
+      if (cg == 0 && ok) {
+#pragma unroll 1
+        for (int g2 = 1; g2 < kColGroups; ++g2) {
+          const float* s2 = sPart + (g2 * kPartialFields) * kBlockM + rloc;
+          Partial o;
+          o.m2 = s2[0 * kBlockM];
+          o.S = s2[1 * kBlockM];
+          o.T2 = s2[2 * kBlockM];
+          o.zmax = s2[3 * kBlockM];
+          o.zarg = __float_as_int(s2[4 * kBlockM]);
+          o.gkey = s2[5 * kBlockM];
+          o.garg = __float_as_int(s2[6 * kBlockM]);
+          partial_merge(pt, o);
+        }
+        const size_t plane = static_cast<size_t>(p.R) * sp.Q;
+        const size_t idx = static_cast<size_t>(row) * sp.Q + q;
+        float* part = p.part;
+        part[0 * plane + idx] = pt.m2;
+        part[1 * plane + idx] = pt.S;
+        part[2 * plane + idx] = pt.T2;
+        part[3 * plane + idx] = pt.zmax;
+        part[4 * plane + idx] = __int_as_float(pt.zarg);
+        part[5 * plane + idx] = pt.gkey;
+        part[6 * plane + idx] = __int_as_float(pt.garg);
+      }
+      epilogue_sync();
     }
   }
 
+  // Both CTAs stay resident until the pair is done: the leader's MMAs read
+  // the peer's shared memory and the peer arrives on the leader's barriers.
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();
   tc_fence_after();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     __syncwarp();
-    tmem_dealloc(tmem_base, 2 * kBlockN);
+    tmem_dealloc_pair(tmem_base, 2 * kBlockN);
   }
 }
 
-HeadSplit head_split(int R, int V, int d, int num_sms) {
+int head_max_pairs() {
+  static int cached = -1;
+  if (cached > 0) return cached;
+  cudaError_t e = cudaFuncSetAttribute(head_sampler_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kHeadSmemBytes);
+  if (e != cudaSuccess) return -1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(kHeadThreads, 1, 1);
+  cfg.dynamicSmemBytes = kHeadSmemBytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, head_sampler_kernel, &cfg) != cudaSuccess || n < 1) return -1;
+  cached = n;
+  return cached;
+}
+
+HeadSplit head_split(int R, int V, int d, int max_pairs) {
   HeadSplit s;
-  s.MT = R / kBlockM;
+  s.MT = R / kPairM;
   s.NT = V / kBlockN;
   s.KB = d / kBlockK;
   const long long quads = static_cast<long long>(s.MT) * (s.NT / 4);
-  if (s.NT % 4 == 0 && quads >= 8LL * num_sms) {
-    s.Q = s.NT / 4;  // units of 4 vocabulary tiles, many per CTA
+  if (s.NT % 4 == 0 && quads >= 8LL * max_pairs) {
+    s.Q = s.NT / 4;  // units of 4 vocabulary tiles, many per pair
   } else {
-    int q = num_sms / s.MT;
+    int q = max_pairs / s.MT;
     if (q < 1) q = 1;
     if (q > s.NT) q = s.NT;
-    s.Q = q;  // about one unit per CTA
+    s.Q = q;  // about one unit per pair
   }
   s.units = s.MT * s.Q;
-  s.grid = s.units < num_sms ? s.units : num_sms;
+  s.pairs = s.units < max_pairs ? s.units : max_pairs;
+  s.grid = 2 * s.pairs;
   return s;
 }
 
 cudaError_t launch_head(const CUtensorMap& tmA, const CUtensorMap& tmB, const HeadParams& p,
                         cudaStream_t stream) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(head_sampler_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kHeadSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  if (head_max_pairs() < 1) return cudaErrorInvalidConfiguration;
   head_sampler_kernel<<<p.split.grid, kHeadThreads, kHeadSmemBytes, stream>>>(tmA, tmB, p);
   return cudaGetLastError();
 }

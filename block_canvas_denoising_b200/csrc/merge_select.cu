@@ -1,7 +1,7 @@
 // merge_select.cu -- cross-tile merge of the head's partials, then the
 // per-canvas entropy-bounded selection, renoise and stop test.
 //
-// Each CTA merges the partial records of 32 rows (8 threads per row, fixed
+// Each CTA merges the partial records of 8 rows (a warp per row, fixed
 // order), writes entropy / sampled / argmax of those rows and takes a ticket
 // on its canvas; the CTA that takes the last ticket of a canvas runs the
 // per-canvas step for all 256 slots:
@@ -25,48 +25,10 @@ namespace dg {
 
 namespace {
 
-constexpr int kRowsPerCta = 32;
-constexpr int kPartsPerRow = 8;
+constexpr int kRowsPerCta = 8;  // one warp per row
 
-struct Acc {
-  float m2, S, T2, zmax;
-  int zarg;
-  float gkey;
-  int garg;
-};
-
-DG_DEV void acc_init(Acc& a) {
-  a.m2 = -1.0e30f;
-  a.S = 0.f;
-  a.T2 = 0.f;
-  a.zmax = -FLT_MAX;
-  a.zarg = INT_MAX;
-  a.gkey = -FLT_MAX;
-  a.garg = INT_MAX;
-}
-
-// Merge b into a.  Softmax: m = max(m_a, m_b), S = sum_i S_i 2^(m_i - m),
-// T2 = sum_i (T2_i + (m_i - m) S_i) 2^(m_i - m).  Argmax and Gumbel key: the
-// larger value wins, ties to the lower vocabulary index.
-DG_DEV void acc_merge(Acc& a, const Acc& b) {
-  const float m = fmaxf(a.m2, b.m2);
-  const float da = a.m2 - m, db = b.m2 - m;
-  const float sa = exp2f(da), sb = exp2f(db);
-  a.T2 = (a.T2 + da * a.S) * sa + (b.T2 + db * b.S) * sb;
-  a.S = a.S * sa + b.S * sb;
-  a.m2 = m;
-  if (b.zmax > a.zmax || (b.zmax == a.zmax && b.zarg < a.zarg)) {
-    a.zmax = b.zmax;
-    a.zarg = b.zarg;
-  }
-  if (b.gkey > a.gkey || (b.gkey == a.gkey && b.garg < a.garg)) {
-    a.gkey = b.gkey;
-    a.garg = b.garg;
-  }
-}
-
-DG_DEV Acc acc_load(const float* part, size_t plane, size_t idx) {
-  Acc a;
+DG_DEV Partial partial_load(const float* part, size_t plane, size_t idx) {
+  Partial a;
   a.m2 = __ldcg(part + 0 * plane + idx);
   a.S = __ldcg(part + 1 * plane + idx);
   a.T2 = __ldcg(part + 2 * plane + idx);
@@ -77,32 +39,44 @@ DG_DEV Acc acc_load(const float* part, size_t plane, size_t idx) {
   return a;
 }
 
+DG_DEV Partial partial_shfl_down(const Partial& a, int off) {
+  Partial o;
+  o.m2 = __shfl_down_sync(0xffffffffu, a.m2, off);
+  o.S = __shfl_down_sync(0xffffffffu, a.S, off);
+  o.T2 = __shfl_down_sync(0xffffffffu, a.T2, off);
+  o.zmax = __shfl_down_sync(0xffffffffu, a.zmax, off);
+  o.zarg = __shfl_down_sync(0xffffffffu, a.zarg, off);
+  o.gkey = __shfl_down_sync(0xffffffffu, a.gkey, off);
+  o.garg = __shfl_down_sync(0xffffffffu, a.garg, off);
+  return o;
+}
+
 }  // namespace
 
 __global__ void __launch_bounds__(256)
 merge_select_kernel(const __grid_constant__ MergeParams p) {
-  __shared__ Acc s_acc[kPartsPerRow][kRowsPerCta];
   __shared__ unsigned long long s_key[256];
   __shared__ float s_h[256];
   __shared__ double s_red[8];
   __shared__ int s_last;
 
   const int t = threadIdx.x;
-  const int r_local = t & (kRowsPerCta - 1);
-  const int part_id = t >> 5;
-  const int row = blockIdx.x * kRowsPerCta + r_local;
-  const size_t plane = static_cast<size_t>(p.P) * p.R;
+  const int warp = t >> 5;
+  const int lane = t & 31;
+  const int row = blockIdx.x * kRowsPerCta + warp;
+  const size_t plane = static_cast<size_t>(p.R) * p.P;
 
-  // ---- merge partials of this row: thread part_id takes p = part_id, +8, ...
-  Acc a;
-  acc_init(a);
-  for (int q = part_id; q < p.P; q += kPartsPerRow)
-    acc_merge(a, acc_load(p.part, plane, static_cast<size_t>(q) * p.R + row));
-  s_acc[part_id][r_local] = a;
-  __syncthreads();
-  if (part_id == 0) {
+  // ---- merge the P partial records of this row: lane j takes j, j+32, ...;
+  // then a fixed tree over the lanes (lane i absorbs lane i + off)
+  Partial a;
+  partial_init(a);
+  for (int q = lane; q < p.P; q += 32) partial_merge(a, partial_load(p.part, plane, static_cast<size_t>(row) * p.P + q));
 #pragma unroll
-    for (int i = 1; i < kPartsPerRow; ++i) acc_merge(a, s_acc[i][r_local]);
+  for (int off = 16; off > 0; off >>= 1) {
+    const Partial o = partial_shfl_down(a, off);
+    if (lane < off) partial_merge(a, o);
+  }
+  if (lane == 0) {
     // H = ln S - ln2 T2 / S, clamped at 0 (the exact value is >= 0)
     float H = logf(a.S) - kLn2 * a.T2 / a.S;
     H = fmaxf(H, 0.0f);

@@ -184,6 +184,16 @@ dg_status dg_denoise_loop(const dg_shape* shape, const dg_params* params,
 
 /* ---- diagnostics (no counterpart on the pages; used by the tests) ---- */
 
+/* Text of the last CUDA runtime error met by a call on this host thread
+ * ("" if none); static thread-local storage, valid until the next call. */
+const char* dg_last_error_message(void);
+
+/* Profiling hook: while set (per host thread), every step records
+ * ev_start / ev_stop (cudaEvent_t handles, created by the caller) on its
+ * stream immediately before and after the fused head kernel, so its device
+ * time can be measured inside a running workload.  NULL, NULL clears it. */
+dg_status dg_set_head_events(void* ev_start, void* ev_stop);
+
 /* Self test of the device-side bounded wait: launches one kernel that waits
  * on a barrier nothing ever arrives at, gives up after limit_ns
  * nanoseconds, latches the fault in the workspace and returns normally.
@@ -193,10 +203,11 @@ dg_status dg_selftest_bounded_wait(uint64_t limit_ns, void* workspace, size_t ws
                                    void* stream);
 
 /* For n Philox words (device uint32 [n]) write the specified float32
- * Gumbel noise g32 = -L(-L(u)) (device float [n]) and the log2 of the
- * approximate Exp(1) variable the sampler's screening pass uses (device
- * float [n]), so tests can compare both with the oracle and bound the
- * approximation over every possible input. */
+ * Gumbel noise g32 = -L(-L(u)) (device float [n]) and the approximate
+ * lg2(E / ln 2), E = -ln u, that the sampler's screening pass uses (device
+ * float [n]; its noise is -ln(ln 2) - ln 2 * lg2(E / ln 2)), so tests can
+ * compare both with the oracle and bound the approximation over every
+ * possible input. */
 dg_status dg_debug_gumbel(const uint32_t* words, int32_t n, float* g_exact, float* lg2e_approx,
                           void* stream);
 
