@@ -16,7 +16,7 @@ import numpy as np
 
 __all__ = ["DGError", "Params", "lib", "workspace_size", "Workspace", "denoise_step",
            "debug_logits", "device_status", "denoise_loop", "debug_gumbel",
-           "selftest_bounded_wait", "set_head_events", "STATUS", "E_BF16", "E_FP8_E4M3"]
+           "selftest_bounded_wait", "set_head_events", "denoise_step_noalloc", "STATUS", "E_BF16", "E_FP8_E4M3"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdg.so")
@@ -93,6 +93,8 @@ def lib() -> ctypes.CDLL:
         L.dg_selftest_bounded_wait.argtypes = [ctypes.c_uint64, P, ctypes.c_size_t, P]
         L.dg_debug_gumbel.argtypes = [P, ctypes.c_int32, P, P, P]
         L.dg_set_head_events.argtypes = [P, P]
+        L.dg_denoise_step_noalloc.argtypes = step_args + [P]
+        L.dg_denoise_step_noalloc.restype = ctypes.c_int
         L.dg_last_error_message.restype = ctypes.c_char_p
         for name in ("dg_workspace_init", "dg_denoise_step", "dg_debug_logits", "dg_device_status",
                      "dg_denoise_loop", "dg_selftest_bounded_wait", "dg_debug_gumbel",
@@ -180,6 +182,29 @@ def denoise_step(h, E, step_idx, has_prev, canvas, prev_argmax, accept, entropy,
     sequences of length B."""
     _step_call("dg_denoise_step", h, E, step_idx, has_prev, canvas, prev_argmax, accept, entropy,
                sampled, argmax, stop, ws, params, e_scale, active, None, stream)
+
+
+def denoise_step_noalloc(h, E, step_idx, has_prev, canvas, prev_argmax, accept, entropy, sampled,
+                         argmax, stop, params: Params = Params(), e_scale=None, active=None,
+                         stream=None) -> None:
+    """``dg_denoise_step_noalloc``: the same step without a caller workspace,
+    for callers that cannot allocate device memory (the scratch is a fixed
+    8 MiB array inside the library; calls must not overlap on the GPU)."""
+    B = int(len(step_idx))
+    R, d = h.shape
+    V = E.shape[0]
+    e_dtype = E_BF16 if e_scale is None else E_FP8_E4M3
+    shp = _shape(B, d, V, e_dtype, L=R // max(B, 1))
+    prm = params.c()
+    ks = _host(step_idx, np.int32)
+    hp = _host(has_prev, np.uint8)
+    act = None if active is None else _host(active, np.uint8)
+    _check(lib().dg_denoise_step_noalloc(
+        ctypes.byref(shp), ctypes.byref(prm), _ptr(h), _ptr(E), _ptr(e_scale),
+        ks.ctypes.data_as(ctypes.c_void_p), hp.ctypes.data_as(ctypes.c_void_p),
+        None if act is None else act.ctypes.data_as(ctypes.c_void_p),
+        _ptr(canvas), _ptr(prev_argmax), _ptr(accept), _ptr(entropy), _ptr(sampled),
+        _ptr(argmax), _ptr(stop), _stream(stream)), "dg_denoise_step_noalloc")
 
 
 def debug_logits(h, E, step_idx, has_prev, canvas, prev_argmax, accept, entropy, sampled, argmax,

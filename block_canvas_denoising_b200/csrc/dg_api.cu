@@ -223,6 +223,10 @@ dg_status run_step(const StepArgs& a) {
 
 }  // namespace
 
+void set_last_error_message(const char* msg) {
+  snprintf(t_last_error, sizeof(t_last_error), "%s", msg);
+}
+
 WsLayout ws_layout(const dg_shape& s, int max_pairs) {
   WsLayout w;
   const int R = s.B * s.L;

@@ -90,6 +90,9 @@ struct WsLayout {
 };
 WsLayout ws_layout(const dg_shape& s, int max_pairs);
 
+// Text returned by dg_last_error_message() on this host thread.
+void set_last_error_message(const char* msg);
+
 cudaError_t launch_head(const CUtensorMap& tmA, const CUtensorMap& tmB, const HeadParams& p,
                         cudaStream_t stream);
 cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream);

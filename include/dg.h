@@ -182,6 +182,33 @@ dg_status dg_denoise_loop(const dg_shape* shape, const dg_params* params,
                           int32_t* argmax, int32_t* stop,
                           void* workspace, size_t ws_bytes, void* stream);
 
+/* dg_denoise_step_noalloc -- dg_denoise_step for callers that cannot
+ * allocate device memory for a workspace: a serving runtime that has carved
+ * up the whole GPU for its own pools, or code that must not call the CUDA
+ * allocator (which can synchronise the device) where it runs steps.  The
+ * pages have no counterpart; this is an interface convenience.
+ *
+ * Same arguments and results as dg_denoise_step, without workspace and
+ * ws_bytes.  The scratch lives in a fixed 8 MiB array of the library's own
+ * device memory, held on every GPU that loads the library until the process
+ * exits.  Shapes needing more (dg_workspace_size() > 8 MiB; on a 148-SM B200
+ * at d = 2816, V = 262,144 that is B > 4) return DG_ERR_WORKSPACE before
+ * anything is launched, with the sizes in dg_last_error_message().  The
+ * first call on a device looks the array's device address up once (the
+ * runtime may initialise the context then), so make it before any stream
+ * capture.  Every call uses the same array: calls that overlap on the GPU
+ * (other streams, other threads) race and must be serialised by the caller.
+ * Each call clears the parts that must start at zero (fault latch, tickets)
+ * on `stream`.  A device-side timeout latches in the array and is cleared
+ * by the next call; it is not reported to the caller. */
+dg_status dg_denoise_step_noalloc(const dg_shape* shape, const dg_params* params,
+                                  const void* h, const void* E, const float* e_scale,
+                                  const int32_t* step_idx, const uint8_t* has_prev,
+                                  const uint8_t* active,
+                                  int32_t* canvas, int32_t* prev_argmax,
+                                  uint8_t* accept, float* entropy, int32_t* sampled,
+                                  int32_t* argmax, int32_t* stop, void* stream);
+
 /* ---- diagnostics (no counterpart on the pages; used by the tests) ---- */
 
 /* Text of the last CUDA runtime error met by a call on this host thread
