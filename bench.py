@@ -205,6 +205,23 @@ def threads_used() -> int:
 
 
 # ---------------------------------------------------------------------------
+# multi-rank plumbing (replicas: no data-path collective)
+# ---------------------------------------------------------------------------
+def rank_seeds(rank: int) -> tuple[int, int]:
+    """(hidden-state seed, Philox seed) of a rank: every rank runs its own
+    canvas against the same embedder (seed 1)."""
+    return 2 + 1000 * rank, 1234 + rank
+
+
+def reduce_max(values, dist, device=None):
+    """Element-wise max of a list of floats over all ranks (no-op alone)."""
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if dist is not None and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
 def init_dist():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -272,8 +289,9 @@ def main():
     dg.lib()
 
     # ---- inputs: one canvas per rank; the embedder is shared model weights
+    h_seed, philox_seed = rank_seeds(rank)
     E_bits = synth.embedder_normal(V, D, seed=1)
-    h_bits = synth.hidden_normal(B, L, D, seed=2 + 1000 * rank)
+    h_bits = synth.hidden_normal(B, L, D, seed=h_seed)
     E = torch.from_numpy(E_bits.view(np.int16)).view(torch.bfloat16).cuda()
     h = torch.from_numpy(h_bits.view(np.int16)).view(torch.bfloat16).cuda()
     R = B * L
@@ -285,7 +303,7 @@ def main():
                amax=torch.zeros(R, dtype=torch.int32, device="cuda"),
                stop=torch.zeros(B, dtype=torch.int32, device="cuda"))
     ws = dg.Workspace(B, D, V)
-    params = dg.Params(seed=1234 + rank)
+    params = dg.Params(seed=philox_seed)
     stream = torch.cuda.current_stream()
 
     def step(i, h_in):
@@ -350,10 +368,7 @@ def main():
     assert dg.device_status(ws) == 0
 
     # max over ranks
-    t = torch.tensor([total_ms, head_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, head_ms = float(t[0]), float(t[1])
+    total_ms, head_ms = reduce_max([total_ms, head_ms], dist, "cuda")
     ms_per_step = total_ms / args.steps
     value = world * B * L / (ms_per_step / 1e3)
 
@@ -379,11 +394,10 @@ def main():
         outs["stop"].copy_(dev["stop"], non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    et = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device="cuda")
+    (e2e_total,) = reduce_max([e0.elapsed_time(e1)], dist, "cuda")
     if world > 1:
-        dist.all_reduce(et, op=dist.ReduceOp.MAX)
         dist.barrier()
-    e2e_ms = float(et[0]) / K2
+    e2e_ms = e2e_total / K2
     e2e_value = world * B * L / (e2e_ms / 1e3)
 
     if rank == 0:

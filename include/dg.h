@@ -18,7 +18,7 @@
  *   [Press]  "Google DiffusionGemma generates 256 tokens in parallel and
  *            self-corrects", section "What DiffusionGemma does" (every
  *            position re-evaluated each step; low-confidence positions are
- *            randomised; the settled block's remaining tokens are locked).
+ *            randomised; once the block settles its open positions are fixed).
  *
  * Conventions for every entry point:
  *   - Tensors are DEVICE pointers owned by the caller unless marked "host".
@@ -162,7 +162,8 @@ typedef int (*dg_hidden_fn)(int32_t k, const int32_t* canvas, void* h_out,
  * one dg_denoise_step runs on every still-active canvas, the B stop flags
  * are read back (one device->host copy per step).  A canvas that stops, or
  * reaches k = max_steps-1, commits: every slot takes that step's sampled
- * token ([Press] "remaining tokens are locked") and the canvas is frozen.
+ * token ([Press]: the settled block's open positions are fixed) and the
+ * canvas is frozen.
  *
  *   h_buf        bf16 [B*L, d] device buffer handed to hidden_fn.
  *   canvas       int32 [B*L] in/out: the committed canvas on return.

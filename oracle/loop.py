@@ -4,7 +4,7 @@
 stop early when the canvas-mean entropy is under 0.005 and two consecutive
 predictions agree.  [Report] Figure 4: the denoising loop refines the canvas
 until it is clean.  [Press] "What DiffusionGemma does": when the block has
-settled, the remaining tokens are locked -- read here as: at the stopping
+settled, its still-open positions get fixed -- read here as: at the stopping
 step (or the last allowed step) every slot takes that step's sampled token.
 Each canvas stops on its own; a stopped canvas is frozen.
 

@@ -94,8 +94,8 @@ def decode_e4m3(bits) -> np.ndarray:
 def temperature(k: int, tau0: float = TAU0, tau1: float = TAU1, max_steps: int = MAX_STEPS) -> float:
     """Linear schedule from tau0 at step 0 to tau1 at step N-1.
 
-    [Docs] temperature-schedule row: "linear 0.8 -> 0.4", high early, low at
-    the end; [Report] Figure 9: a larger N gives milder annealing, so the
+    [Docs] temperature-schedule row: a linear decrease from 0.8 to 0.4, hot
+    at the start and cool at the end; [Report] Figure 9: a larger N gives milder annealing, so the
     schedule spans the N steps.  For N = 1 the single step uses tau0.
     """
     if not 0 <= k < max_steps:
