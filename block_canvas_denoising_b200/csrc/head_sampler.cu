@@ -476,6 +476,10 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
   }
 
+  // Let the dependent merge kernel launch; it waits (griddepcontrol.wait)
+  // for this grid's completion before reading the partial records.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
   // Both CTAs stay resident until the pair is done: the leader's MMAs read
   // the peer's shared memory and the peer arrives on the leader's barriers.
   tc_fence_before();

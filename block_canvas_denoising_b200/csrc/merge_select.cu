@@ -66,6 +66,10 @@ merge_select_kernel(const __grid_constant__ MergeParams p) {
   const int row = blockIdx.x * kRowsPerCta + warp;
   const size_t plane = static_cast<size_t>(p.R) * p.P;
 
+  // Launched as a programmatic dependent of the head kernel: wait until its
+  // partial records are complete and visible.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
   // ---- merge the P partial records of this row: lane j takes j, j+32, ...;
   // then a fixed tree over the lanes (lane i absorbs lane i + off)
   Partial a;
@@ -113,14 +117,20 @@ merge_select_kernel(const __grid_constant__ MergeParams p) {
   s_key[s] = key;
   s_h[s] = H;
   __syncthreads();
-  double csum = 0.0;
-  int rank = 0;
-#pragma unroll 8
-  for (int i = 0; i < 256; ++i) {
-    const unsigned long long ki = s_key[i];
-    if (ki <= key) csum += static_cast<double>(s_h[i]);
-    rank += (ki < key) ? 1 : 0;
+  // four independent running sums over i = j mod 4, added in a fixed order
+  double cs[4] = {0.0, 0.0, 0.0, 0.0};
+  int rk[4] = {0, 0, 0, 0};
+#pragma unroll 4
+  for (int i = 0; i < 256; i += 4) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const unsigned long long ki = s_key[i + j];
+      if (ki <= key) cs[j] += static_cast<double>(s_h[i + j]);
+      rk[j] += (ki < key) ? 1 : 0;
+    }
   }
+  const double csum = (cs[0] + cs[1]) + (cs[2] + cs[3]);
+  const int rank = (rk[0] + rk[1]) + (rk[2] + rk[3]);
   const bool accepted = (csum <= p.entropy_bound) || (rank == 0);
 
   // ---- renoise
@@ -154,9 +164,19 @@ merge_select_kernel(const __grid_constant__ MergeParams p) {
 }
 
 cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream) {
-  const int grid = p.R / kRowsPerCta;
-  merge_select_kernel<<<grid, 256, 0, stream>>>(p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.R / kRowsPerCta, 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  // programmatic dependent launch: the launch overlaps the head kernel's
+  // tail; griddepcontrol.wait in the kernel orders the data
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, merge_select_kernel, p);
 }
 
 }  // namespace dg
