@@ -26,7 +26,7 @@ E_FP8_E4M3 = 1
 
 STATUS = {0: "DG_OK", 1: "DG_ERR_INVALID_ARG", 2: "DG_ERR_UNSUPPORTED_SHAPE", 3: "DG_ERR_WORKSPACE",
           4: "DG_ERR_RANGE", 5: "DG_ERR_CUDA", 6: "DG_ERR_TIMEOUT", 7: "DG_ERR_CALLBACK",
-          8: "DG_ERR_NO_DEVICE"}
+          8: "DG_ERR_NO_DEVICE", 9: "DG_ERR_VALUE"}
 
 
 class DGError(RuntimeError):

@@ -16,7 +16,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libdg.so")
 
-SOURCES = ["dg_api.cu", "head_sampler.cu", "merge_select.cu", "diagnostics.cu", "noalloc.cu"]
+SOURCES = ["dg_api.cu", "head_sampler.cu", "hidden_split.cu", "merge_select.cu", "diagnostics.cu", "noalloc.cu"]
 HEADERS = ["dg_device.cuh", "dg_internal.h"]
 
 

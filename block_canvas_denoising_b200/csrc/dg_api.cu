@@ -60,7 +60,7 @@ dg_status check_shape(const dg_shape* s) {
   if (s->B < 1 || s->B > DG_MAX_B || s->L != 256 || s->d < kBlockK || s->d % kBlockK != 0 ||
       s->V < kBlockN || s->V % kBlockN != 0)
     return DG_ERR_UNSUPPORTED_SHAPE;
-  if (s->e_dtype != DG_E_BF16) return DG_ERR_UNSUPPORTED_SHAPE;
+  if (s->e_dtype != DG_E_BF16 && s->e_dtype != DG_E_FP8_E4M3) return DG_ERR_UNSUPPORTED_SHAPE;
   return DG_OK;
 }
 
@@ -90,17 +90,18 @@ float inv_tau_of(const dg_params& p, int k) {
   return static_cast<float>(1.0 / tau);
 }
 
-bool encode_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
-                    uint32_t box_inner, uint32_t box_rows) {
+// 2-D tensor map over a row-major [rows, inner] matrix with elements of
+// `dtype` (`esize` bytes); box = box_inner x box_rows elements.
+bool encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t esize, CUtensorMapSwizzle swizzle,
+               const void* base, uint64_t inner, uint64_t rows, uint32_t box_inner, uint32_t box_rows) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {inner, rows};
-  cuuint64_t strides[1] = {inner * 2};
+  cuuint64_t strides[1] = {inner * esize};
   cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -136,11 +137,14 @@ dg_status run_step(const StepArgs& a) {
       !a.entropy || !a.sampled || !a.argmax || !a.stop || !a.workspace)
     return DG_ERR_INVALID_ARG;
   if (!aligned16(a.h) || !aligned16(a.E) || !aligned16(a.workspace)) return DG_ERR_INVALID_ARG;
+  const bool fp8 = s.e_dtype == DG_E_FP8_E4M3;
+  // the per-row scale belongs to the FP8 embedder only
+  if (fp8 ? (a.e_scale == nullptr || !aligned16(a.e_scale)) : a.e_scale != nullptr) return DG_ERR_INVALID_ARG;
   if (a.logits != nullptr && !aligned16(a.logits)) return DG_ERR_INVALID_ARG;
   for (int b = 0; b < s.B; ++b)
     if (a.step_idx[b] < 0 || a.step_idx[b] >= pr.max_steps) return DG_ERR_RANGE;
   if (device_sms() <= 0) return DG_ERR_NO_DEVICE;
-  const int pairs = head_max_pairs();
+  const int pairs = head_max_pairs(fp8);
   if (pairs <= 0) {
     snprintf(t_last_error, sizeof(t_last_error), "no CTA pair of the head kernel fits on this device");
     return DG_ERR_CUDA;
@@ -160,15 +164,34 @@ dg_status run_step(const StepArgs& a) {
     cps[b].active = (a.active == nullptr || a.active[b]) ? 1 : 0;
   }
 
-  // TMA boxes: one CTA's share of a stage.  The kernel's expect-tx byte
-  // counts and shared-memory slots are sized from the same constants.
-  static_assert(kAStageBytes == kBlockK * kBlockM * 2, "A box / stage mismatch");
-  static_assert(kBStageBytes == kBlockK * kHalfN * 2, "B box / stage mismatch");
-  CUtensorMap tmA, tmB;
-  if (!encode_2d_bf16(&tmA, a.h, static_cast<uint64_t>(s.d), static_cast<uint64_t>(R), kBlockK, kBlockM))
-    return DG_ERR_CUDA;
-  if (!encode_2d_bf16(&tmB, a.E, static_cast<uint64_t>(s.d), static_cast<uint64_t>(s.V), kBlockK, kHalfN))
-    return DG_ERR_CUDA;
+  // TMA boxes: one CTA's share of a stage, 128 rows x 128 bytes of K (the
+  // 128-byte swizzle span); the kernel's expect-tx byte counts and shared-
+  // memory slots are sized from the same constants.  K beyond d reads as 0.
+  static_assert(kTileBytes == kBlockK * 2 * kBlockM && kTileBytes == kBlockKFp8 * 1 * kHalfN,
+                "TMA box / stage tile mismatch");
+  CUtensorMap tmA, tmA2, tmB;
+  if (fp8) {
+    // h -> h1 + h2 (E4M3) with a power-of-two row scale, in the workspace
+    uint8_t* h1 = wsb + ws.h1_off;
+    uint8_t* h2 = wsb + ws.h2_off;
+    if (!cuda_ok(launch_hidden_split(a.h, h1, h2, reinterpret_cast<float*>(wsb + ws.rinv_off), R, s.d,
+                                     reinterpret_cast<uint32_t*>(wsb + ws.err_off), a.stream),
+                 "hidden-state split launch"))
+      return DG_ERR_CUDA;
+    const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
+    if (!encode_2d(&tmA, U8, 1, SW, h1, s.d, R, kBlockKFp8, kBlockM) ||
+        !encode_2d(&tmA2, U8, 1, SW, h2, s.d, R, kBlockKFp8, kBlockM) ||
+        !encode_2d(&tmB, U8, 1, SW, a.E, s.d, s.V, kBlockKFp8, kHalfN))
+      return DG_ERR_CUDA;
+  } else {
+    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
+    if (!encode_2d(&tmA, BF, 2, SW, a.h, s.d, R, kBlockK, kBlockM) ||
+        !encode_2d(&tmB, BF, 2, SW, a.E, s.d, s.V, kBlockK, kHalfN))
+      return DG_ERR_CUDA;
+    tmA2 = tmA;  // unused by the bf16 head
+  }
 
   HeadParams hp;
   memset(&hp, 0, sizeof(hp));
@@ -176,7 +199,7 @@ dg_status run_step(const StepArgs& a) {
   hp.d = s.d;
   hp.V = s.V;
   hp.B = s.B;
-  hp.split = head_split(R, s.V, s.d, pairs);
+  hp.split = head_split(R, s.V, s.d, pairs, fp8 ? kBlockKFp8 : kBlockK);
   hp.seed_lo = static_cast<uint32_t>(pr.seed & 0xFFFFFFFFull);
   hp.seed_hi = static_cast<uint32_t>(pr.seed >> 32);
   // Philox4x32-10 round keys: key + i * (0x9E3779B9, 0xBB67AE85), mod 2^32
@@ -185,6 +208,7 @@ dg_status run_step(const StepArgs& a) {
     hp.rk1[i] = hp.seed_hi + static_cast<uint32_t>(i) * 0xBB67AE85u;
   }
   hp.e_scale = a.e_scale;
+  hp.row_inv = fp8 ? reinterpret_cast<const float*>(wsb + ws.rinv_off) : nullptr;
   hp.part = reinterpret_cast<float*>(wsb + ws.part_off);
   hp.err = reinterpret_cast<uint32_t*>(wsb + ws.err_off);
   hp.logits_out = a.logits;
@@ -193,7 +217,7 @@ dg_status run_step(const StepArgs& a) {
 
   if (t_head_ev_start != nullptr && cudaEventRecord(t_head_ev_start, a.stream) != cudaSuccess)
     return DG_ERR_CUDA;
-  if (!cuda_ok(launch_head(tmA, tmB, hp, a.stream), "head kernel launch")) return DG_ERR_CUDA;
+  if (!cuda_ok(launch_head(fp8, tmA, tmA2, tmB, hp, a.stream), "head kernel launch")) return DG_ERR_CUDA;
   if (t_head_ev_stop != nullptr && cudaEventRecord(t_head_ev_stop, a.stream) != cudaSuccess)
     return DG_ERR_CUDA;
 
@@ -230,12 +254,17 @@ void set_last_error_message(const char* msg) {
 WsLayout ws_layout(const dg_shape& s, int max_pairs) {
   WsLayout w;
   const int R = s.B * s.L;
-  const HeadSplit sp = head_split(R, s.V, s.d, max_pairs);
+  const bool fp8 = s.e_dtype == DG_E_FP8_E4M3;
+  const HeadSplit sp = head_split(R, s.V, s.d, max_pairs, fp8 ? kBlockKFp8 : kBlockK);
   w.P = sp.Q;
   w.err_off = 0;
   w.tickets_off = kAlign;
   w.part_off = align_up(w.tickets_off + sizeof(uint32_t) * static_cast<size_t>(s.B));
-  w.total = align_up(w.part_off + sizeof(float) * kPartialFields * static_cast<size_t>(w.P) * R);
+  const size_t hsz = fp8 ? static_cast<size_t>(R) * s.d : 0;  // one E4M3 term of h
+  w.h1_off = align_up(w.part_off + sizeof(float) * kPartialFields * static_cast<size_t>(w.P) * R);
+  w.h2_off = align_up(w.h1_off + hsz);
+  w.rinv_off = align_up(w.h2_off + hsz);
+  w.total = align_up(w.rinv_off + (fp8 ? sizeof(float) * static_cast<size_t>(R) : 0));
   return w;
 }
 
@@ -267,6 +296,7 @@ const char* dg_error_string(dg_status s) {
     case DG_ERR_TIMEOUT: return "device-side wait timed out";
     case DG_ERR_CALLBACK: return "hidden-state callback failed";
     case DG_ERR_NO_DEVICE: return "no sm_100 device";
+    case DG_ERR_VALUE: return "input value outside the supported range";
   }
   return "unknown status";
 }
@@ -274,7 +304,7 @@ const char* dg_error_string(dg_status s) {
 size_t dg_workspace_size(const dg_shape* shape) {
   if (check_shape(shape) != DG_OK) return 0;
   if (device_sms() <= 0) return 0;
-  const int pairs = head_max_pairs();
+  const int pairs = head_max_pairs(shape->e_dtype == DG_E_FP8_E4M3);
   if (pairs <= 0) return 0;
   return ws_layout(*shape, pairs).total;
 }
@@ -319,7 +349,9 @@ dg_status dg_device_status(void* workspace, size_t ws_bytes, void* stream) {
   if (err != 0) {
     if (cudaMemsetAsync(workspace, 0, sizeof(err), st) != cudaSuccess) return DG_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return DG_ERR_CUDA;
-    return DG_ERR_TIMEOUT;
+    if (err & ~static_cast<uint32_t>(kErrHiddenRange)) return DG_ERR_TIMEOUT;
+    set_last_error_message("FP8 head: a hidden-state value is not finite");
+    return DG_ERR_VALUE;
   }
   return DG_OK;
 }

@@ -21,6 +21,7 @@ enum : uint32_t {
   kErrWaitMmaAcc = 1u << 2,       // MMA issuer gave up waiting for a drained accumulator
   kErrWaitEpilogue = 1u << 3,     // epilogue gave up waiting for a finished tile
   kErrSelftest = 1u << 4,         // the bounded-wait self test ran out (expected)
+  kErrHiddenRange = 1u << 5,      // FP8 head: a hidden-state value is not finite
 };
 
 // ---------------------------------------------------------------------------
@@ -66,15 +67,34 @@ DG_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The same test with acquire semantics at cluster scope: for barriers that
+// the peer CTA's threads arrive on (release.cluster) after writing memory
+// the waiter then reads.
+DG_DEV bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase of parity `parity` to complete, for at most `limit_ns`
 // nanoseconds of %globaltimer.  Returns false if the limit ran out.
+template <bool kClusterScope = false>
 DG_DEV bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+  auto test = [&]() {
+    return kClusterScope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+  };
+  if (test()) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+      if (test()) return true;
     if (global_timer_ns() - t0 > limit_ns) return false;
   }
 }
@@ -209,6 +229,17 @@ DG_DEV void tc_mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, ui
       : "memory");
 }
 
+// Pair MMA with E4M3 operands (K = 32 per instruction), f32 accumulate.
+DG_DEV void tc_mma_e4m3_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, f32 accumulate.
 DG_DEV void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                         uint32_t accumulate) {
@@ -242,6 +273,12 @@ DG_DEV uint64_t smem_desc_k_sw128(uint32_t saddr) {
 __host__ __device__ constexpr uint32_t instr_desc_bf16_f32(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// kind::f8f6f4 with E4M3 A and B (format code 0 in [7,10) and [10,13)),
+// f32 accumulator, both K-major.
+__host__ __device__ constexpr uint32_t instr_desc_e4m3_f32(int M, int N) {
+  return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 // Issue a load of 32 consecutive f32 columns of this thread's TMEM lane

@@ -18,19 +18,31 @@ constexpr int kPairM = 256;                       // rows per pair tile
 constexpr int kBlockM = 128;                      // rows per CTA
 constexpr int kBlockN = 256;                      // vocabulary columns per tile
 constexpr int kHalfN = 128;                       // E rows staged per CTA
-constexpr int kBlockK = 64;
-constexpr int kStages = 6;
+constexpr int kBlockK = 64;                       // bf16 K per stage: one 128-byte row
+constexpr int kBlockKFp8 = 128;                   // E4M3 K per stage: one 128-byte row
 constexpr int kEpiWarps = 16;                     // 4 column groups x 4 lane quarters
 constexpr int kColGroups = kEpiWarps / 4;         // 64 columns each
 constexpr int kProducerWarp = kEpiWarps;          // warp 16
 constexpr int kMmaWarp = kEpiWarps + 1;           // warp 17
 constexpr int kHeadThreads = (kEpiWarps + 2) * 32;
-constexpr int kAStageBytes = kBlockM * kBlockK * 2;
-constexpr int kBStageBytes = kHalfN * kBlockK * 2;
+constexpr int kTileBytes = 128 * 128;             // 128 rows x 128 B, 128-byte swizzle
 constexpr int kPartialFields = 7;                 // m2, S, T2, zmax, zarg, gkey, garg
 // per-unit exchange of the column groups' partials inside a CTA
 constexpr int kPartSmemBytes = kColGroups * kBlockM * kPartialFields * 4;
-constexpr int kHeadSmemBytes = kStages * (kAStageBytes + kBStageBytes) + 1024 + 256 + kPartSmemBytes;
+
+// Pipeline of the two head variants.  bf16 embedder: a stage holds one h
+// tile and one E tile of 64 K.  E4M3 embedder: a stage holds the two E4M3
+// terms of h (h1, h2) and one tile of E codes, 128 K each.
+template <bool kFp8>
+struct HeadCfg {
+  static constexpr int kStages = kFp8 ? 4 : 6;
+  static constexpr int kBlockKElems = kFp8 ? kBlockKFp8 : kBlockK;
+  static constexpr int kATiles = kFp8 ? 2 : 1;
+  static constexpr int kStageBytes = (kATiles + 1) * kTileBytes;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256 + kPartSmemBytes;
+};
+static_assert(HeadCfg<false>::kSmemBytes <= 232448, "bf16 head exceeds 227 KB of shared memory");
+static_assert(HeadCfg<true>::kSmemBytes <= 232448, "FP8 head exceeds 227 KB of shared memory");
 constexpr uint64_t kDefaultWaitNs = 4000000000ull;
 
 // Per-canvas step data, filled on the host.
@@ -54,7 +66,8 @@ struct HeadParams {
   int32_t R, d, V, B;
   HeadSplit split;
   uint32_t seed_lo, seed_hi;
-  const float* e_scale;  // per-vocabulary-row scale (FP8) or null
+  const float* e_scale;  // FP8: per-vocabulary-row scale, else null
+  const float* row_inv;  // FP8: 2^-k_r, the inverse of h's per-row split scale, else null
   float* part;           // partial records, kPartialFields planes of [R][Q]
   uint32_t* err;         // device fault latch
   float* logits_out;     // optional raw logits [R, V]
@@ -80,21 +93,32 @@ struct MergeParams {
   CanvasParam cp[DG_MAX_B];
 };
 
-HeadSplit head_split(int R, int V, int d, int max_pairs);
-int head_max_pairs();
+// kblock: K elements per stage (kBlockK, or kBlockKFp8 for the FP8 head);
+// KB = ceil(d / kblock), the last stage's K tail read as zeros.
+HeadSplit head_split(int R, int V, int d, int max_pairs, int kblock);
+int head_max_pairs(bool fp8);
 
 // Workspace layout (byte offsets), see dg_workspace_size().
 struct WsLayout {
-  size_t err_off, tickets_off, part_off, total;
+  size_t err_off, tickets_off, part_off, h1_off, h2_off, rinv_off, total;
   int P;
 };
+// FP8 embedder only: h1, h2 E4M3 [R, d] (the two terms of h's split) and
+// rinv float [R] (2^-k_r).
 WsLayout ws_layout(const dg_shape& s, int max_pairs);
 
 // Text returned by dg_last_error_message() on this host thread.
 void set_last_error_message(const char* msg);
 
-cudaError_t launch_head(const CUtensorMap& tmA, const CUtensorMap& tmB, const HeadParams& p,
-                        cudaStream_t stream);
+// bf16 head: tmA = h bf16 [R, d], tmB = E bf16 [V, d] (tmA2 unused).
+// FP8 head:  tmA = h1, tmA2 = h2 (E4M3 [R, d]), tmB = E codes E4M3 [V, d].
+cudaError_t launch_head(bool fp8, const CUtensorMap& tmA, const CUtensorMap& tmA2, const CUtensorMap& tmB,
+                        const HeadParams& p, cudaStream_t stream);
+// Split each row r of h (bf16 [R, d], d a multiple of 8, 16-byte aligned)
+// into E4M3 terms h1 + h2 = h * 2^k_r and write rinv[r] = 2^-k_r; latches
+// kErrHiddenRange in *err if some h is not finite.
+cudaError_t launch_hidden_split(const void* h, uint8_t* h1, uint8_t* h2, float* rinv, int R, int d,
+                                uint32_t* err, cudaStream_t stream);
 cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream);
 cudaError_t launch_wait_selftest(uint32_t* err, uint64_t limit_ns, cudaStream_t stream);
 cudaError_t launch_gumbel_probe(const uint32_t* words, int n, float* g_exact, float* lg2e_approx,

@@ -16,16 +16,27 @@
 //
 // The kernel runs as CTA pairs (clusters of 2) on the tcgen05 cta_group::2
 // path: the pair computes 256 rows x 256 vocabulary columns per tile, the
-// leader CTA issuing 256x256x16 bf16 MMAs over both CTAs' shared memory;
-// each CTA holds its 128-row half of the tile in its own TMEM.
+// leader CTA issuing 256x256xK MMAs over both CTAs' shared memory; each CTA
+// holds its 128-row half of the tile in its own TMEM.
 //
-// Warp roles (320 threads per CTA, one CTA per SM, persistent):
-//   warp 0      TMA producer: this CTA's halves of the h and E tiles into a
-//               6-stage shared-memory ring (completion on the leader's barrier).
-//   warp 1      TMEM allocator; in the leader, the MMA issuer.
-//   warps 2..9  epilogue: warp w reads TMEM lane quarter w % 4 and column
-//               half (w - 2) / 4 of each tile; two accumulators alternate
-//               so the epilogue of tile t overlaps the MMAs of tile t + 1.
+// Warp roles (576 threads, one CTA per SM, persistent):
+//   warps 0..15  epilogue: warp w reads TMEM lane quarter w % 4 and 64-column
+//                group w / 4 of each tile; two accumulators alternate so the
+//                epilogue of tile t overlaps the MMAs of tile t + 1.
+//   warp 16      TMA producer: this CTA's halves of the h and E tiles into a
+//                shared-memory ring (completion on the leader's barrier).
+//   warp 17      TMEM allocator; in the leader, the MMA issuer.
+//
+// FP8 embedder (E4M3 codes q with a float32 scale s_v per vocabulary row):
+// the codes go from HBM to the tensor cores untouched (kind::f8f6f4, half
+// the bytes of bf16).  h is split once per step by a small kernel into two
+// E4M3 terms with a power-of-two row scale, h[r] * 2^k_r = h1[r] + h2[r],
+// and every K step issues the two MMAs h1 . q^T and h2 . q^T into the same
+// accumulator -- at twice the bf16 rate, the same tensor time as one bf16
+// MMA.  The epilogue forms z = (acc * s_v) * 2^-k_r.  The split is exact
+// for every |h| >= 2^-9 max_k |h[r, k]| (8 significant bits in two 4-bit
+// terms); below that its error is at most 2^-10 * 2^-k_r.
+// ([Docs] "DiffusionGemma": the model is served with FP8 weights.)
 #include <float.h>
 #include <limits.h>
 
@@ -192,23 +203,21 @@ DG_DEV void process8(const float (&z)[8], int v0, float inv_tau, float c2, uint3
   }
 }
 
-// Scale (FP8 embedder), optional logits dump, then the group's reductions.
-DG_DEV void epi_group(const uint32_t (&r)[8], int v0, int row, float inv_tau, float c2, uint32_t ctr1,
-                      uint32_t ctr2, uint32_t ctr3, const HeadParams& p, Partial& pt, Screen& sc) {
+// Scales (FP8 embedder: z = (acc * s_v) * rinv, rinv = 2^-k_r), optional
+// logits dump, then the group's reductions.
+template <bool kFp8>
+DG_DEV void epi_group(const uint32_t (&r)[8], int v0, int row, float rinv, float inv_tau, float c2,
+                      uint32_t ctr1, uint32_t ctr2, uint32_t ctr3, const HeadParams& p, Partial& pt,
+                      Screen& sc) {
   float z[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) z[j] = __uint_as_float(r[j]);
-  if (p.e_scale != nullptr) {
+  if (kFp8) {
     const float4* scp = reinterpret_cast<const float4*>(p.e_scale + v0);
     const float4 s0 = __ldg(scp), s1 = __ldg(scp + 1);
-    z[0] = __fmul_rn(z[0], s0.x);
-    z[1] = __fmul_rn(z[1], s0.y);
-    z[2] = __fmul_rn(z[2], s0.z);
-    z[3] = __fmul_rn(z[3], s0.w);
-    z[4] = __fmul_rn(z[4], s1.x);
-    z[5] = __fmul_rn(z[5], s1.y);
-    z[6] = __fmul_rn(z[6], s1.z);
-    z[7] = __fmul_rn(z[7], s1.w);
+    const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) z[j] = __fmul_rn(__fmul_rn(z[j], sv[j]), rinv);
   }
   if (p.logits_out != nullptr) {
     float4* dst = reinterpret_cast<float4*>(p.logits_out + static_cast<size_t>(row) * p.V + v0);
@@ -225,14 +234,20 @@ DG_DEV void epilogue_sync() {
 
 }  // namespace
 
+template <bool kFp8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kHeadThreads, 1)
-head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const __grid_constant__ HeadParams p) {
+head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
+                    const __grid_constant__ CUtensorMap tmB, const __grid_constant__ HeadParams p) {
+  using Cfg = HeadCfg<kFp8>;
+  constexpr int kStages = Cfg::kStages;
+  constexpr int kATiles = Cfg::kATiles;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // stage s: A tile(s) at sA + (s * kATiles + t) * kTileBytes, E tile at sB + s * kTileBytes
   uint8_t* sA = smem;
-  uint8_t* sB = smem + kStages * kAStageBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + kStages * kBStageBytes);
+  uint8_t* sB = smem + kStages * kATiles * kTileBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + kStages * kTileBytes);
+  // barriers: full[S], empty[S], tfull[2], tempty[2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 4);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   // [column group][field][row of the CTA half]
@@ -252,6 +267,7 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 
   if (threadIdx.x == 0) {
     prefetch_tensormap(&tmA);
+    if (kFp8) prefetch_tensormap(&tmA2);
     prefetch_tensormap(&tmB);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(full_bar(s), 1);   // leader's producer arrival + both CTAs' bytes
@@ -295,11 +311,14 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
               break;
             }
             const uint32_t fb = full_bar(stage);
-            if (rank == 0) mbar_arrive_expect_tx(fb, 2 * (kAStageBytes + kBStageBytes));
+            if (rank == 0) mbar_arrive_expect_tx(fb, 2 * Cfg::kStageBytes);
             const uint32_t fb_leader = mapa_shared(fb, 0);
-            tma_load_2d_pair(smem_u32(sA + stage * kAStageBytes), &tmA, fb_leader, kb * kBlockK,
-                             m * kPairM + static_cast<int>(rank) * kBlockM, pol_h);
-            tma_load_2d_pair(smem_u32(sB + stage * kBStageBytes), &tmB, fb_leader, kb * kBlockK,
+            const int kx = kb * Cfg::kBlockKElems;  // 128 B of K: 16-byte aligned
+            const int hrow = m * kPairM + static_cast<int>(rank) * kBlockM;
+            uint8_t* a0 = sA + stage * kATiles * kTileBytes;
+            tma_load_2d_pair(smem_u32(a0), &tmA, fb_leader, kx, hrow, pol_h);
+            if (kFp8) tma_load_2d_pair(smem_u32(a0 + kTileBytes), &tmA2, fb_leader, kx, hrow, pol_h);
+            tma_load_2d_pair(smem_u32(sB + stage * kTileBytes), &tmB, fb_leader, kx,
                              n * kBlockN + static_cast<int>(rank) * kHalfN, pol_e);
             if (++stage == kStages) {
               stage = 0;
@@ -324,7 +343,7 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer (leader)
     if (lane == 0 && rank == 0) {
-      constexpr uint32_t idesc = instr_desc_bf16_f32(kPairM, kBlockN);
+      constexpr uint32_t idesc = kFp8 ? instr_desc_e4m3_f32(kPairM, kBlockN) : instr_desc_bf16_f32(kPairM, kBlockN);
       int stage = 0;
       uint32_t phase = 0;
       int tile = 0;
@@ -335,7 +354,7 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         for (int n = n0; n < n1 && ok; ++n, ++tile) {
           const int acc = tile & 1;
           const uint32_t acc_phase = (tile >> 1) & 1;
-          if (!mbar_wait_bounded(tempty_bar(acc), acc_phase ^ 1u, p.wait_ns)) {
+          if (!mbar_wait_bounded<true>(tempty_bar(acc), acc_phase ^ 1u, p.wait_ns)) {
             latch_error(p.err, kErrWaitMmaAcc);
             ok = false;
             break;
@@ -349,13 +368,20 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
               break;
             }
             tc_fence_after();
-            const uint64_t adesc = smem_desc_k_sw128(smem_u32(sA + stage * kAStageBytes));
-            const uint64_t bdesc = smem_desc_k_sw128(smem_u32(sB + stage * kBStageBytes));
+            const uint64_t adesc = smem_desc_k_sw128(smem_u32(sA + stage * kATiles * kTileBytes));
+            const uint64_t bdesc = smem_desc_k_sw128(smem_u32(sB + stage * kTileBytes));
+            // 32 B of K per instruction (16 bf16 or 32 E4M3): +2 in the
+            // descriptor's 16-byte address field, inside the swizzled rows
 #pragma unroll
-            for (int k16 = 0; k16 < kBlockK / 16; ++k16) {
-              // advance 16 bf16 = 32 B along K inside the swizzled rows
-              tc_mma_bf16_pair(d_tmem, adesc + 2u * k16, bdesc + 2u * k16, idesc,
-                               (kb > 0 || k16 > 0) ? 1u : 0u);
+            for (int k32 = 0; k32 < 4; ++k32) {
+              const uint32_t acc_flag = (kb > 0 || k32 > 0) ? 1u : 0u;
+              if (kFp8) {
+                constexpr uint64_t kTileDesc = kTileBytes >> 4;  // next A tile: h2
+                tc_mma_e4m3_pair(d_tmem, adesc + 2u * k32, bdesc + 2u * k32, idesc, acc_flag);
+                tc_mma_e4m3_pair(d_tmem, adesc + kTileDesc + 2u * k32, bdesc + 2u * k32, idesc, 1u);
+              } else {
+                tc_mma_bf16_pair(d_tmem, adesc + 2u * k32, bdesc + 2u * k32, idesc, acc_flag);
+              }
             }
             tc_commit_pair_mc(empty_bar(stage), 0x3);  // frees the stage in both CTAs
             if (++stage == kStages) {
@@ -384,6 +410,7 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       const int slot = row & 255;
       const CanvasParam cp = p.cp[b];
       const float inv_tau = cp.inv_tau;
+      const float rinv = kFp8 ? __ldg(p.row_inv + row) : 1.0f;
       const float c2 = __fmul_rn(inv_tau, kLog2e);
       const uint32_t ctr1 = static_cast<uint32_t>(slot) | (kPurposeGumbel << 16);
       const uint32_t ctr2 = static_cast<uint32_t>(cp.k);
@@ -417,10 +444,10 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 #pragma unroll 1
         for (int g = 0; g < kGroups; g += 2) {
           tmem_load8_issue(tbase + 8 * (g + 1), rb);
-          epi_group(ra, vbase + 8 * g, row, inv_tau, c2, ctr1, ctr2, ctr3, p, pt, sc);
+          epi_group<kFp8>(ra, vbase + 8 * g, row, rinv, inv_tau, c2, ctr1, ctr2, ctr3, p, pt, sc);
           tmem_load8_wait(rb);
           if (g + 2 < kGroups) tmem_load8_issue(tbase + 8 * (g + 2), ra);
-          epi_group(rb, vbase + 8 * (g + 1), row, inv_tau, c2, ctr1, ctr2, ctr3, p, pt, sc);
+          epi_group<kFp8>(rb, vbase + 8 * (g + 1), row, rinv, inv_tau, c2, ctr1, ctr2, ctr3, p, pt, sc);
           tmem_load8_wait(ra);
           __syncwarp();
         }
@@ -491,16 +518,17 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   }
 }
 
-int head_max_pairs() {
+template <bool kFp8>
+int max_pairs_of() {
   static int cached = -1;
   if (cached > 0) return cached;
-  cudaError_t e = cudaFuncSetAttribute(head_sampler_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       kHeadSmemBytes);
+  constexpr int kSmem = HeadCfg<kFp8>::kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(head_sampler_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return -1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2, 1, 1);
   cfg.blockDim = dim3(kHeadThreads, 1, 1);
-  cfg.dynamicSmemBytes = kHeadSmemBytes;
+  cfg.dynamicSmemBytes = kSmem;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
@@ -509,16 +537,18 @@ int head_max_pairs() {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, head_sampler_kernel, &cfg) != cudaSuccess || n < 1) return -1;
+  if (cudaOccupancyMaxActiveClusters(&n, head_sampler_kernel<kFp8>, &cfg) != cudaSuccess || n < 1) return -1;
   cached = n;
   return cached;
 }
 
-HeadSplit head_split(int R, int V, int d, int max_pairs) {
+int head_max_pairs(bool fp8) { return fp8 ? max_pairs_of<true>() : max_pairs_of<false>(); }
+
+HeadSplit head_split(int R, int V, int d, int max_pairs, int kblock) {
   HeadSplit s;
   s.MT = R / kPairM;
   s.NT = V / kBlockN;
-  s.KB = d / kBlockK;
+  s.KB = (d + kblock - 1) / kblock;
   const long long quads = static_cast<long long>(s.MT) * (s.NT / 4);
   if (s.NT % 4 == 0 && quads >= 8LL * max_pairs) {
     s.Q = s.NT / 4;  // units of 4 vocabulary tiles, many per pair
@@ -534,10 +564,14 @@ HeadSplit head_split(int R, int V, int d, int max_pairs) {
   return s;
 }
 
-cudaError_t launch_head(const CUtensorMap& tmA, const CUtensorMap& tmB, const HeadParams& p,
-                        cudaStream_t stream) {
-  if (head_max_pairs() < 1) return cudaErrorInvalidConfiguration;
-  head_sampler_kernel<<<p.split.grid, kHeadThreads, kHeadSmemBytes, stream>>>(tmA, tmB, p);
+cudaError_t launch_head(bool fp8, const CUtensorMap& tmA, const CUtensorMap& tmA2, const CUtensorMap& tmB,
+                        const HeadParams& p, cudaStream_t stream) {
+  if (head_max_pairs(fp8) < 1) return cudaErrorInvalidConfiguration;
+  if (fp8)
+    head_sampler_kernel<true><<<p.split.grid, kHeadThreads, HeadCfg<true>::kSmemBytes, stream>>>(tmA, tmA2, tmB, p);
+  else
+    head_sampler_kernel<false><<<p.split.grid, kHeadThreads, HeadCfg<false>::kSmemBytes, stream>>>(tmA, tmA2, tmB,
+                                                                                                    p);
   return cudaGetLastError();
 }
 

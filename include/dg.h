@@ -53,7 +53,9 @@ typedef enum {
   DG_ERR_CUDA = 5,             /* a CUDA runtime call failed */
   DG_ERR_TIMEOUT = 6,          /* a device-side bounded wait ran out */
   DG_ERR_CALLBACK = 7,         /* the hidden-state callback returned non-zero */
-  DG_ERR_NO_DEVICE = 8         /* no sm_100 device current */
+  DG_ERR_NO_DEVICE = 8,        /* no sm_100 device current */
+  DG_ERR_VALUE = 9             /* FP8 head: a hidden-state value is not finite
+                                  (found on the device) */
 } dg_status;
 
 typedef enum { DG_E_BF16 = 0, DG_E_FP8_E4M3 = 1 } dg_edtype;
@@ -102,7 +104,15 @@ dg_status dg_workspace_init(void* workspace, size_t ws_bytes, void* stream);
  *   E         embedder [V, d] row-major: bf16, or FP8-E4M3 codes (uint8)
  *             when shape->e_dtype == DG_E_FP8_E4M3.  The tied LM head
  *             ([Report] Table 1) is z = h . E^T (times e_scale[v] for FP8).
- *   e_scale   float [V] per-row dequantisation scale (FP8 only, else NULL).
+ *   e_scale   float [V] per-row dequantisation scale, 16-byte aligned:
+ *             required for FP8, must be NULL for bf16 (DG_ERR_INVALID_ARG).
+ *             The FP8 head computes z[r, v] = e_scale[v] * sum_k h[r,k] q[v,k]
+ *             on E4M3 tensor-core operands: q as given, and h split per row
+ *             into two E4M3 terms with a power-of-two scale 2^k_r
+ *             (h * 2^k_r = h1 + h2), exact for every |h[r,k]| >= 2^-9 *
+ *             max_k |h[r,k]| and within 2^-10 * 2^-k_r below that.  A
+ *             non-finite h latches DG_ERR_VALUE (see dg_device_status) and
+ *             leaves the step's results undefined.
  *   step_idx  HOST int32 [B]: step k of each canvas, 0 <= k < max_steps.
  *             tau_k = tau0 - (tau0 - tau1) * k / (max_steps - 1)
  *             ([Docs] temperature schedule), tau0 for max_steps == 1.
@@ -147,7 +157,8 @@ dg_status dg_debug_logits(const dg_shape* shape, const dg_params* params,
                           void* workspace, size_t ws_bytes, void* stream);
 
 /* Synchronise `stream`, then read and clear the device fault latch of the
- * workspace.  Returns DG_OK, DG_ERR_TIMEOUT or DG_ERR_CUDA. */
+ * workspace.  Returns DG_OK, DG_ERR_TIMEOUT (a bounded wait ran out),
+ * DG_ERR_VALUE (FP8 head: a non-finite h) or DG_ERR_CUDA. */
 dg_status dg_device_status(void* workspace, size_t ws_bytes, void* stream);
 
 /* Hidden-state producer for the loop: writes the bf16 [B*L, d] hidden
@@ -200,8 +211,9 @@ dg_status dg_denoise_loop(const dg_shape* shape, const dg_params* params,
  * capture.  Every call uses the same array: calls that overlap on the GPU
  * (other streams, other threads) race and must be serialised by the caller.
  * Each call clears the parts that must start at zero (fault latch, tickets)
- * on `stream`.  A device-side timeout latches in the array and is cleared
- * by the next call; it is not reported to the caller. */
+ * on `stream`.  A device-side timeout (or, for the FP8 head, a non-finite
+ * h) latches in the array and is cleared by the next call; it is not
+ * reported to the caller. */
 dg_status dg_denoise_step_noalloc(const dg_shape* shape, const dg_params* params,
                                   const void* h, const void* E, const float* e_scale,
                                   const int32_t* step_idx, const uint8_t* has_prev,

@@ -28,16 +28,29 @@ def to_dev_bf16(bits):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
 
 
+def to_dev_fp8(q, s):
+    """E4M3 codes (uint8 [V, d]) and their float32 row scales on the device."""
+    import torch
+    return (torch.from_numpy(np.ascontiguousarray(q, dtype=np.uint8)).cuda(),
+            torch.from_numpy(np.ascontiguousarray(s, dtype=np.float32)).cuda())
+
+
 def run_step(h_bits, E_bits, step_idx, has_prev, prev_argmax, canvas0, params, *,
-             debug=True, active=None):
-    """One step through the C ABI; returns numpy outputs (and logits)."""
+             debug=True, active=None, e_scale=None):
+    """One step through the C ABI; returns numpy outputs (and logits).
+
+    With ``e_scale`` (float32 [V]) ``E_bits`` holds E4M3 codes (uint8) and
+    the FP8 head runs."""
     import torch
     import block_canvas_denoising_b200 as dg
     B = len(step_idx)
     R, d = h_bits.shape
     V = E_bits.shape[0]
     h = to_dev_bf16(h_bits)
-    E = to_dev_bf16(E_bits)
+    if e_scale is None:
+        E, sc, e_dtype = to_dev_bf16(E_bits), None, dg.E_BF16
+    else:
+        (E, sc), e_dtype = to_dev_fp8(E_bits, e_scale), dg.E_FP8_E4M3
     dev = dict(
         canvas=torch.from_numpy(np.asarray(canvas0, np.int32).copy()).cuda(),
         prev_argmax=torch.from_numpy(np.asarray(prev_argmax, np.int32).copy()).cuda(),
@@ -47,17 +60,17 @@ def run_step(h_bits, E_bits, step_idx, has_prev, prev_argmax, canvas0, params, *
         argmax=torch.zeros(R, dtype=torch.int32, device="cuda"),
         stop=torch.full((B,), -1, dtype=torch.int32, device="cuda"),
     )
-    ws = dg.Workspace(B, d, V)
+    ws = dg.Workspace(B, d, V, e_dtype)
     if debug:
         logits = torch.empty((R, V), dtype=torch.float32, device="cuda")
         dg.debug_logits(h, E, step_idx, has_prev, dev["canvas"], dev["prev_argmax"], dev["accept"],
                         dev["entropy"], dev["sampled"], dev["argmax"], dev["stop"], logits, ws,
-                        params, active=active)
+                        params, e_scale=sc, active=active)
     else:
         logits = None
         dg.denoise_step(h, E, step_idx, has_prev, dev["canvas"], dev["prev_argmax"], dev["accept"],
                         dev["entropy"], dev["sampled"], dev["argmax"], dev["stop"], ws, params,
-                        active=active)
+                        e_scale=sc, active=active)
     assert dg.device_status(ws) == 0
     torch.cuda.synchronize()
     out = {k: v.cpu().numpy() for k, v in dev.items()}
@@ -76,12 +89,16 @@ def rows_of(canvases, L=256):
 
 
 def compare_with_oracle(g, h_bits, E_bits, step_idx, has_prev, prev_argmax, params, canvases=None,
-                        L=256, report=None):
-    """Compare device outputs ``g`` with the oracle on the chosen canvases."""
+                        L=256, report=None, e_scale=None):
+    """Compare device outputs ``g`` with the oracle on the chosen canvases.
+
+    With ``e_scale``, ``E_bits`` holds E4M3 codes and the oracle dequantises
+    them (codes times row scale, in float64)."""
     B = len(step_idx)
     canvases = list(range(B)) if canvases is None else list(canvases)
     op = oparams(params)
-    ora = oracle.denoise_step(h_bits, E_bits=E_bits, B=B, L=L, step_idx=step_idx, has_prev=has_prev,
+    emb = dict(E_bits=E_bits) if e_scale is None else dict(q=E_bits, s=e_scale)
+    ora = oracle.denoise_step(h_bits, **emb, B=B, L=L, step_idx=step_idx, has_prev=has_prev,
                               prev_argmax=prev_argmax, params=op, canvases=canvases)
     rows = rows_of(canvases, L)
     n = len(rows)
@@ -91,7 +108,7 @@ def compare_with_oracle(g, h_bits, E_bits, step_idx, has_prev, prev_argmax, para
 
     # logits (on the same rows)
     if "logits" in g:
-        z_or = np.concatenate([oracle.step.logits(h_bits[b * L:(b + 1) * L], E_bits=E_bits)
+        z_or = np.concatenate([oracle.step.logits(h_bits[b * L:(b + 1) * L], **emb)
                                for b in canvases])
         zg = g["logits"][rows].astype(np.float64)
         err = np.abs(zg - z_or).max()

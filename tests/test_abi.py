@@ -46,18 +46,19 @@ def test_default_params_are_serving_defaults(libdg):
 
 
 def test_error_strings(libdg):
-    for code in range(9):
+    for code in range(10):
         assert libdg.dg_error_string(code)
+    assert libdg.dg_error_string(9) != libdg.dg_error_string(99)
 
 
-def _call_step(libdg, B=1, L=256, d=512, V=8192, ks=(0,), e_dtype=0, null=False):
+def _call_step(libdg, B=1, L=256, d=512, V=8192, ks=(0,), e_dtype=0, null=False, e_scale=None):
     shp = dg._Shape(B, L, d, V, e_dtype)
     prm = dg.Params().c()
     ksa = np.asarray(ks, np.int32)
     hp = np.zeros(max(B, 1), np.uint8)
     fake = ctypes.c_void_p(0 if null else 256)   # never dereferenced: checks fail first
     P = [fake] * 9
-    return libdg.dg_denoise_step(ctypes.byref(shp), ctypes.byref(prm), fake, fake, None,
+    return libdg.dg_denoise_step(ctypes.byref(shp), ctypes.byref(prm), fake, fake, e_scale,
                                  ksa.ctypes.data_as(ctypes.c_void_p), hp.ctypes.data_as(ctypes.c_void_p),
                                  None, *P[:7], fake, ctypes.c_size_t(1 << 30), None)
 
@@ -74,6 +75,15 @@ def test_null_and_range_checks(libdg):
     assert _call_step(libdg, null=True) == 1
     assert _call_step(libdg, ks=(48,)) == 4
     assert _call_step(libdg, ks=(-1,)) == 4
+
+
+def test_embedder_scale_checks(libdg):
+    # the per-row scale is required for the FP8 embedder, refused for bf16,
+    # and must be 16-byte aligned (all found before any device work)
+    assert _call_step(libdg, e_dtype=1) == 1
+    assert _call_step(libdg, e_dtype=0, e_scale=ctypes.c_void_p(512)) == 1
+    assert _call_step(libdg, e_dtype=1, e_scale=ctypes.c_void_p(520)) == 1
+    assert _call_step(libdg, e_dtype=2, e_scale=ctypes.c_void_p(512)) == 2
 
 
 def test_workspace_size_zero_for_bad_shape(libdg):
