@@ -212,6 +212,7 @@ dg_status run_step(const StepArgs& a) {
   hp.part = reinterpret_cast<float*>(wsb + ws.part_off);
   hp.err = reinterpret_cast<uint32_t*>(wsb + ws.err_off);
   hp.logits_out = a.logits;
+  hp.row_rec = reinterpret_cast<uint32_t*>(wsb + ws.rec_off);
   hp.wait_ns = kDefaultWaitNs;
   memcpy(hp.cp, cps, sizeof(cps));
 
@@ -236,6 +237,7 @@ dg_status run_step(const StepArgs& a) {
   mp.accept = a.accept;
   mp.stop = a.stop;
   mp.tickets = reinterpret_cast<uint32_t*>(wsb + ws.tickets_off);
+  mp.row_rec = hp.row_rec;
   mp.seed_lo = hp.seed_lo;
   mp.seed_hi = hp.seed_hi;
   mp.entropy_bound = pr.entropy_bound;
@@ -259,7 +261,9 @@ WsLayout ws_layout(const dg_shape& s, int max_pairs) {
   w.P = sp.Q;
   w.err_off = 0;
   w.tickets_off = kAlign;
-  w.part_off = align_up(w.tickets_off + sizeof(uint32_t) * static_cast<size_t>(s.B));
+  w.rec_off = align_up(w.tickets_off + sizeof(uint32_t) * static_cast<size_t>(s.B));
+  w.part_off = align_up(w.rec_off + sizeof(uint32_t) * static_cast<size_t>(R));
+  w.zero_prefix = w.part_off;
   const size_t hsz = fp8 ? static_cast<size_t>(R) * s.d : 0;  // one E4M3 term of h
   w.h1_off = align_up(w.part_off + sizeof(float) * kPartialFields * static_cast<size_t>(w.P) * R);
   w.h2_off = align_up(w.h1_off + hsz);

@@ -5,6 +5,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <float.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -567,6 +568,22 @@ DG_DEV float lg2_exp1_approx(uint32_t r) {
 
 // C0 = -ln(ln 2): g = C0 - ln2 * lg2(E2).
 constexpr float kGumbelC0 = 0.36651292058166432f;
+
+// Order-preserving map of a (non-NaN) float onto uint32: a < b <=> enc(a) <
+// enc(b); 0 is never produced and stands for "no key yet".
+DG_DEV uint32_t key_order_enc(float k) {
+  const uint32_t b = __float_as_uint(k);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+DG_DEV float key_order_dec(uint32_t e) {
+  if (e == 0u) return -FLT_MAX;
+  return __uint_as_float((e & 0x80000000u) ? (e & 0x7FFFFFFFu) : ~e);
+}
+
+// The largest specified noise, g32 at the largest u = 1 - 2^-24 (g32 is
+// nondecreasing in the word; both facts are checked against the oracle over
+// all 2^23 inputs).
+constexpr float kGumbelMaxNoise = 16.635532f;
 
 // |approx key - specified key| <= kGumbelApproxErr + rounding of the keys.
 constexpr float kGumbelApproxErr = 1.0e-5f;

@@ -29,6 +29,8 @@ constexpr int kTileBytes = 128 * 128;             // 128 rows x 128 B, 128-byte 
 constexpr int kPartialFields = 7;                 // m2, S, T2, zmax, zarg, gkey, garg
 // per-unit exchange of the column groups' partials inside a CTA
 constexpr int kPartSmemBytes = kColGroups * kBlockM * kPartialFields * 4;
+// best screening key seen so far by each column group, per row of the CTA
+constexpr int kRecSmemBytes = kColGroups * kBlockM * 4;
 
 // Pipeline of the two head variants.  bf16 embedder: a stage holds one h
 // tile and one E tile of 64 K.  E4M3 embedder: a stage holds the two E4M3
@@ -39,7 +41,7 @@ struct HeadCfg {
   static constexpr int kBlockKElems = kFp8 ? kBlockKFp8 : kBlockK;
   static constexpr int kATiles = kFp8 ? 2 : 1;
   static constexpr int kStageBytes = (kATiles + 1) * kTileBytes;
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256 + kPartSmemBytes;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256 + kPartSmemBytes + kRecSmemBytes;
 };
 static_assert(HeadCfg<false>::kSmemBytes <= 232448, "bf16 head exceeds 227 KB of shared memory");
 static_assert(HeadCfg<true>::kSmemBytes <= 232448, "FP8 head exceeds 227 KB of shared memory");
@@ -71,6 +73,7 @@ struct HeadParams {
   float* part;           // partial records, kPartialFields planes of [R][Q]
   uint32_t* err;         // device fault latch
   float* logits_out;     // optional raw logits [R, V]
+  uint32_t* row_rec;     // [R] best screening key per row so far (ordered encoding, 0 = none)
   uint64_t wait_ns;
   uint32_t rk0[10], rk1[10];  // Philox round keys of the seed
   CanvasParam cp[DG_MAX_B];
@@ -87,6 +90,7 @@ struct MergeParams {
   uint8_t* accept;
   int32_t* stop;
   uint32_t* tickets;  // [B], self-resetting
+  uint32_t* row_rec;  // [R] the head's per-row key records, cleared here for the next step
   uint32_t seed_lo, seed_hi;
   double entropy_bound;
   double stop_entropy;
@@ -100,7 +104,8 @@ int head_max_pairs(bool fp8);
 
 // Workspace layout (byte offsets), see dg_workspace_size().
 struct WsLayout {
-  size_t err_off, tickets_off, part_off, h1_off, h2_off, rinv_off, total;
+  size_t err_off, tickets_off, rec_off, part_off, h1_off, h2_off, rinv_off, total;
+  size_t zero_prefix;  // bytes from the start that must be zero before a step (latch, tickets, records)
   int P;
 };
 // FP8 embedder only: h1, h2 E4M3 [R, d] (the two terms of h's split) and

@@ -109,9 +109,11 @@ DG_DEV void top2(float& a1, float& a2, float b1, float b2) {
 }
 
 // Eight consecutive logits of one row: z[0..7] are vocabulary v0 .. v0+7.
+// thr: the best screening key any column group of this row has reached in
+// the current unit (a lower bound on the row's winning key, up to eps).
 DG_DEV void process8(const float (&z)[8], int v0, float inv_tau, float c2, uint32_t ctr1,
                      uint32_t ctr2, uint32_t ctr3, const uint32_t (&rk0)[10], const uint32_t (&rk1)[10],
-                     Partial& pt, Screen& sc) {
+                     float thr, Partial& pt, Screen& sc) {
   // ---- group max, argmax of z (ties to the lower index; groups arrive in
   // increasing v)
   const float m01 = fmaxf(z[0], z[1]), m23 = fmaxf(z[2], z[3]);
@@ -153,6 +155,16 @@ DG_DEV void process8(const float (&z)[8], int v0, float inv_tau, float c2, uint3
   }
 
   // ---- Gumbel-max screen (branch-free except for rare near-ties)
+  // Group bound: g32 is nondecreasing in the Philox word and x = fl(z inv_tau)
+  // in z, so no key of the group exceeds fl(fl(gmax inv_tau) + g32(max word)).
+  // When even that bound is clearly below the best key already known for the
+  // row, no element of the group can win or tie: skip it (first with the
+  // largest possible noise, before any Philox work, then with the group's).
+  // The margin covers the screen's error on both keys and the index packing.
+  const float lim = fmaxf(sc.K1a, thr);
+  const float lim_eps = lim - 2.0f * screen_eps(lim);
+  const float x0max = __fmaf_rn(gmax, inv_tau, kGumbelC0);
+  if (x0max + (kGumbelMaxNoise + 1e-3f - kGumbelC0) < lim_eps) return;
   const uint32_t cb = static_cast<uint32_t>(v0) >> 2;
   uint32_t w[8];
   {
@@ -164,6 +176,10 @@ DG_DEV void process8(const float (&z)[8], int v0, float inv_tau, float c2, uint3
       w[l] = wa[l];
       w[4 + l] = wb[l];
     }
+  }
+  {
+    const uint32_t wm = max(max(max(w[0], w[1]), max(w[2], w[3])), max(max(w[4], w[5]), max(w[6], w[7])));
+    if (__fmaf_rn(lg2_exp1_approx(wm), -kLn2, x0max) < lim_eps) return;
   }
   float kp[8];
 #pragma unroll
@@ -206,8 +222,8 @@ DG_DEV void process8(const float (&z)[8], int v0, float inv_tau, float c2, uint3
 // Scales (FP8 embedder: z = (acc * s_v) * rinv, rinv = 2^-k_r), optional
 // logits dump, then the group's reductions.
 template <bool kFp8>
-DG_DEV void epi_group(const uint32_t (&r)[8], int v0, int row, float rinv, float inv_tau, float c2,
-                      uint32_t ctr1, uint32_t ctr2, uint32_t ctr3, const HeadParams& p, Partial& pt,
+DG_DEV void epi_group(const uint32_t* r, int v0, int row, float rinv, float inv_tau, float c2,
+                      uint32_t ctr1, uint32_t ctr2, uint32_t ctr3, float thr, const HeadParams& p, Partial& pt,
                       Screen& sc) {
   float z[8];
 #pragma unroll
@@ -224,7 +240,7 @@ DG_DEV void epi_group(const uint32_t (&r)[8], int v0, int row, float rinv, float
     dst[0] = make_float4(z[0], z[1], z[2], z[3]);
     dst[1] = make_float4(z[4], z[5], z[6], z[7]);
   }
-  process8(z, v0, inv_tau, c2, ctr1, ctr2, ctr3, p.rk0, p.rk1, pt, sc);
+  process8(z, v0, inv_tau, c2, ctr1, ctr2, ctr3, p.rk0, p.rk1, thr, pt, sc);
 }
 
 // Named barrier over the epilogue warps only (barrier 1).
@@ -252,6 +268,8 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   // [column group][field][row of the CTA half]
   float* sPart = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);
+  // [column group][row of the CTA half]: best screening key of the unit so far
+  volatile float* sRec = sPart + kColGroups * kPartialFields * kBlockM;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -284,6 +302,7 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     tmem_alloc_pair(smem_u32(tmem_slot), 2 * kBlockN);
     tmem_relinquish_pair();
   }
+  if (threadIdx.x < kEpiWarps * 32) sRec[threadIdx.x] = -FLT_MAX;
   tc_fence_before();
   cluster_sync_all();
   tc_fence_after();
@@ -419,6 +438,8 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       partial_init(pt);
       Screen sc;
       screen_reset(sc);
+      uint32_t grec = __ldcg(p.row_rec + row);
+      float published = -FLT_MAX;
       for (int n = n0; n < n1; ++n, ++tile) {
         const int acc = tile & 1;
         const uint32_t acc_phase = (tile >> 1) & 1;
@@ -437,6 +458,13 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                static_cast<uint32_t>(acc * kBlockN + cg * (kBlockN / kColGroups));
         const int vbase = n * kBlockN + cg * (kBlockN / kColGroups);
+        // best key this row has reached so far: in this CTA's column groups
+        // (shared memory) and in every CTA (the global record, read one tile
+        // ahead to hide its latency); stale values are lower, hence safe
+        const float thr = fmaxf(fmaxf(fmaxf(sRec[0 * kBlockM + rloc], sRec[1 * kBlockM + rloc]),
+                                      fmaxf(sRec[2 * kBlockM + rloc], sRec[3 * kBlockM + rloc])),
+                                key_order_dec(grec));
+        grec = __ldcg(p.row_rec + row);
         uint32_t ra[8], rb[8];
         __syncwarp();
         tmem_load8_issue(tbase, ra);
@@ -444,12 +472,17 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 #pragma unroll 1
         for (int g = 0; g < kGroups; g += 2) {
           tmem_load8_issue(tbase + 8 * (g + 1), rb);
-          epi_group<kFp8>(ra, vbase + 8 * g, row, rinv, inv_tau, c2, ctr1, ctr2, ctr3, p, pt, sc);
+          epi_group<kFp8>(ra, vbase + 8 * g, row, rinv, inv_tau, c2, ctr1, ctr2, ctr3, thr, p, pt, sc);
           tmem_load8_wait(rb);
           if (g + 2 < kGroups) tmem_load8_issue(tbase + 8 * (g + 2), ra);
-          epi_group<kFp8>(rb, vbase + 8 * (g + 1), row, rinv, inv_tau, c2, ctr1, ctr2, ctr3, p, pt, sc);
+          epi_group<kFp8>(rb, vbase + 8 * (g + 1), row, rinv, inv_tau, c2, ctr1, ctr2, ctr3, thr, p, pt, sc);
           tmem_load8_wait(ra);
           __syncwarp();
+        }
+        sRec[cg * kBlockM + rloc] = sc.K1a;
+        if (sc.K1a > published) {
+          atomicMax(p.row_rec + row, key_order_enc(sc.K1a));
+          published = sc.K1a;
         }
         tc_fence_before();
         __syncwarp();
@@ -499,6 +532,9 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         part[5 * plane + idx] = pt.gkey;
         part[6 * plane + idx] = __int_as_float(pt.garg);
       }
+      // the next unit may cover other rows: its records start afresh (no
+      // epilogue warp reads them between the two barriers)
+      sRec[cg * kBlockM + rloc] = -FLT_MAX;
       epilogue_sync();
     }
   }

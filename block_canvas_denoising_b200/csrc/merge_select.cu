@@ -81,6 +81,7 @@ merge_select_kernel(const __grid_constant__ MergeParams p) {
     if (lane < off) partial_merge(a, o);
   }
   if (lane == 0) {
+    p.row_rec[row] = 0u;  // the head's key record of this row starts empty next step
     // H = ln S - ln2 T2 / S, clamped at 0 (the exact value is >= 0)
     float H = logf(a.S) - kLn2 * a.T2 / a.S;
     H = fmaxf(H, 0.0f);

@@ -76,10 +76,12 @@ extern "C" dg_status dg_denoise_step_noalloc(const dg_shape* shape, const dg_par
   void* ws = nullptr;
   dg_status st = scratch_address(&ws);
   if (st != DG_OK) return st;
-  // The array keeps the previous call's contents.  The fault latch and the
-  // per-canvas tickets must start at zero (everything else is written before
-  // it is read), so clear them on the caller's stream; this does not allocate.
-  const size_t zero_bytes = 256 + sizeof(uint32_t) * static_cast<size_t>(shape->B);
+  // The array keeps the previous call's contents.  The fault latch, the
+  // per-canvas tickets and the per-row key records must start at zero
+  // (everything else is written before it is read), so clear them on the
+  // caller's stream; this does not allocate.
+  const size_t zero_bytes =
+      dg::ws_layout(*shape, dg::head_max_pairs(shape->e_dtype == DG_E_FP8_E4M3)).zero_prefix;
   if (cudaMemsetAsync(ws, 0, zero_bytes, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DG_ERR_CUDA;
   return dg_denoise_step(shape, params, h, E, e_scale, step_idx, has_prev, active, canvas, prev_argmax, accept,
                          entropy, sampled, argmax, stop, ws, kNoAllocScratchBytes, stream);
