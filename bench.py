@@ -10,6 +10,11 @@ The embedder (1.48 GB) is far larger than the 126 MB L2, so every step
 streams it from HBM; no flush is needed.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                  [--e-dtype fp8]
+
+``--e-dtype fp8`` times the FP8-E4M3 embedder variant instead (E quantised
+per row to E4M3 codes with a float32 scale, h still bf16); the default line
+is the bf16 workload.
 
 For N > 1 launch with torch.distributed.run; each rank runs its own canvas
 (replicas, no data-path collective): weak scaling.  ``--impl reference``
@@ -52,6 +57,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e-dtype", default="bf16", choices=("bf16", "fp8"))
     return ap.parse_args()
 
 
@@ -292,7 +298,15 @@ def main():
     h_seed, philox_seed = rank_seeds(rank)
     E_bits = synth.embedder_normal(V, D, seed=1)
     h_bits = synth.hidden_normal(B, L, D, seed=h_seed)
-    E = torch.from_numpy(E_bits.view(np.int16)).view(torch.bfloat16).cuda()
+    fp8 = args.e_dtype == "fp8"
+    if fp8:
+        q_codes, e_scale_np = synth.quantize_e4m3_rows(E_bits)
+        E = torch.from_numpy(q_codes).cuda()
+        e_scale = torch.from_numpy(e_scale_np).cuda()
+        del q_codes
+    else:
+        E = torch.from_numpy(E_bits.view(np.int16)).view(torch.bfloat16).cuda()
+        e_scale = None
     h = torch.from_numpy(h_bits.view(np.int16)).view(torch.bfloat16).cuda()
     R = B * L
     dev = dict(canvas=torch.zeros(R, dtype=torch.int32, device="cuda"),
@@ -302,13 +316,14 @@ def main():
                samp=torch.zeros(R, dtype=torch.int32, device="cuda"),
                amax=torch.zeros(R, dtype=torch.int32, device="cuda"),
                stop=torch.zeros(B, dtype=torch.int32, device="cuda"))
-    ws = dg.Workspace(B, D, V)
+    ws = dg.Workspace(B, D, V, dg.E_FP8_E4M3 if fp8 else dg.E_BF16)
     params = dg.Params(seed=philox_seed)
     stream = torch.cuda.current_stream()
 
     def step(i, h_in):
         dg.denoise_step(h_in, E, [KS[i % 3]], [1 if i > 0 else 0], dev["canvas"], dev["prev"],
-                        dev["acc"], dev["ent"], dev["samp"], dev["amax"], dev["stop"], ws, params)
+                        dev["acc"], dev["ent"], dev["samp"], dev["amax"], dev["stop"], ws, params,
+                        e_scale=e_scale)
 
     def timed_region(K):
         ev_h = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -402,19 +417,25 @@ def main():
 
     if rank == 0:
         pk, pk_kind = peaks()
-        alg_bytes = V * D * 2 + R * D * 2
+        e_bytes = 1 if fp8 else 2
+        alg_bytes = V * D * e_bytes + R * D * 2
         achieved = alg_bytes / (head_ms / 1e3) / 1e9
-        traffic, _ = recorded_traffic()
+        traffic, _ = recorded_traffic() if not fp8 else (None, None)
+        # FP8: two E4M3 MMAs per K step at twice the bf16 rate (nominal
+        # ratio): the same tensor time as 2 R D V bf16 flops
         flops = 2.0 * R * D * V
         line = {
             "metric": METRIC, "value": value, "unit": "slots/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3 (h split in two E4M3 terms)" if fp8 else "bf16",
             "data": "synthetic",
-            "config": {"workload": "B=1 canvas (256 slots) per GPU, d=2816, V=262144, bf16 h and E, "
-                                   "k cycling 0/23/47",
+            "config": {"workload": ("B=1 canvas (256 slots) per GPU, d=2816, V=262144, bf16 h, "
+                                    "E4M3 embedder with per-row float32 scale, k cycling 0/23/47") if fp8 else
+                                   ("B=1 canvas (256 slots) per GPU, d=2816, V=262144, bf16 h and E, "
+                                    "k cycling 0/23/47"),
                        "global_batch": world * B, "seq_len": L, "parallelism": f"replicas x{world}",
-                       "l2": "inputs larger than L2 (E = 1.48 GB streamed each step)"},
+                       "l2": "inputs larger than L2 (E = %.2f GB streamed each step)" % (V * D * e_bytes / 1e9)},
             "us_per_step": ms_per_step * 1e3,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
@@ -427,9 +448,9 @@ def main():
             "clocks": clocks,
             "e2e": {"value": e2e_value, "unit": "slots/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": 2 * args.steps,
+            "gpu_launches": (3 if fp8 else 2) * args.steps,
         }
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and not fp8:
             t_cpu = oracle_canvas_step(h_bits, E_bits, 0)
             line["cpu_baseline"] = {"value": L / t_cpu, "unit": "slots/s", "cores": threads_used(),
                                     "kind": "oracle",

@@ -87,3 +87,20 @@ def test_gumbel_transform_accuracy():
     # monotone in u, as -ln(-ln u) is
     order = np.argsort(u)
     assert np.all(np.diff(g32[order]) >= 0)
+
+
+def test_gumbel_noise_is_nondecreasing_over_every_word_and_its_maximum():
+    # The sampler's group bound relies on two facts about the specified noise
+    # g32: it never decreases as the Philox word grows, and its largest value
+    # (u = 1 - 2^-24) is the constant the CUDA screen uses.  Both are checked
+    # here over all 2^23 distinct uniforms.
+    import os
+    import re
+    r = (np.arange(1 << 23, dtype=np.uint64) << np.uint64(9)).astype(np.uint32)
+    g = flog.gumbel_f32(flog.uniform_f32(r))
+    assert np.all(np.diff(g) >= 0)
+    src = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                            "block_canvas_denoising_b200", "csrc", "dg_device.cuh")).read()
+    m = re.search(r"kGumbelMaxNoise\s*=\s*([0-9.]+)f", src)
+    assert m is not None
+    assert np.float32(m.group(1)) == g.max()
