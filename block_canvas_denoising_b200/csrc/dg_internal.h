@@ -22,8 +22,13 @@ constexpr int kBlockK = 64;                       // bf16 K per stage: one 128-b
 constexpr int kBlockKFp8 = 128;                   // E4M3 K per stage: one 128-byte row
 constexpr int kEpiWarps = 16;                     // 4 column groups x 4 lane quarters
 constexpr int kColGroups = kEpiWarps / 4;         // 64 columns each
-constexpr int kProducerWarp = kEpiWarps;          // warp 16
-constexpr int kMmaWarp = kEpiWarps + 1;           // warp 17
+// The MMA issuer is warp 0 and the TMA producer warp 1: the warp schedulers
+// favour lower warps, and the single thread that feeds the tensor core must
+// not wait behind the epilogue warps sharing its scheduler.  The epilogue
+// warps 2..17 cover every (TMEM lane quarter = warp % 4, column group) pair.
+constexpr int kMmaWarp = 0;
+constexpr int kProducerWarp = 1;
+constexpr int kEpiWarp0 = 2;
 constexpr int kHeadThreads = (kEpiWarps + 2) * 32;
 constexpr int kTileBytes = 128 * 128;             // 128 rows x 128 B, 128-byte swizzle
 constexpr int kPartialFields = 7;                 // m2, S, T2, zmax, zarg, gkey, garg

@@ -20,12 +20,12 @@
 // holds its 128-row half of the tile in its own TMEM.
 //
 // Warp roles (576 threads, one CTA per SM, persistent):
-//   warps 0..15  epilogue: warp w reads TMEM lane quarter w % 4 and 64-column
-//                group w / 4 of each tile; two accumulators alternate so the
-//                epilogue of tile t overlaps the MMAs of tile t + 1.
-//   warp 16      TMA producer: this CTA's halves of the h and E tiles into a
+//   warp 0       TMEM allocator; in the leader, the MMA issuer.
+//   warp 1       TMA producer: this CTA's halves of the h and E tiles into a
 //                shared-memory ring (completion on the leader's barrier).
-//   warp 17      TMEM allocator; in the leader, the MMA issuer.
+//   warps 2..17  epilogue: warp w reads TMEM lane quarter w % 4 and 64-column
+//                group (w - 2) / 4 of each tile; two accumulators alternate so
+//                the epilogue of tile t overlaps the MMAs of tile t + 1.
 //
 // FP8 embedder (E4M3 codes q with a float32 scale s_v per vocabulary row):
 // the codes go from HBM to the tensor cores untouched (kind::f8f6f4, half
@@ -302,7 +302,7 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     tmem_alloc_pair(smem_u32(tmem_slot), 2 * kBlockN);
     tmem_relinquish_pair();
   }
-  if (threadIdx.x < kEpiWarps * 32) sRec[threadIdx.x] = -FLT_MAX;
+  if (threadIdx.x >= kEpiWarp0 * 32) sRec[threadIdx.x - kEpiWarp0 * 32] = -FLT_MAX;
   tc_fence_before();
   cluster_sync_all();
   tc_fence_after();
@@ -361,8 +361,19 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer (leader)
+    // One thread feeds the tensor core while 4 epilogue warps share its
+    // scheduler, so its loop is kept short: descriptors and barrier
+    // addresses advance by constant 32-bit steps per stage.
     if (lane == 0 && rank == 0) {
       constexpr uint32_t idesc = kFp8 ? instr_desc_e4m3_f32(kPairM, kBlockN) : instr_desc_bf16_f32(kPairM, kBlockN);
+      const uint64_t a_desc0 = smem_desc_k_sw128(smem_u32(sA));
+      const uint64_t b_desc0 = smem_desc_k_sw128(smem_u32(sB));
+      const uint32_t a_hi = static_cast<uint32_t>(a_desc0 >> 32), b_hi = static_cast<uint32_t>(b_desc0 >> 32);
+      const uint32_t a_lo0 = static_cast<uint32_t>(a_desc0), b_lo0 = static_cast<uint32_t>(b_desc0);
+      constexpr uint32_t kAStep = (kATiles * kTileBytes) >> 4;  // descriptor units of 16 B
+      constexpr uint32_t kBStep = kTileBytes >> 4;
+      const uint32_t full0 = full_bar(0), empty0 = empty_bar(0);
+      uint32_t a_lo = a_lo0, b_lo = b_lo0, fb = full0, eb = empty0;
       int stage = 0;
       uint32_t phase = 0;
       int tile = 0;
@@ -381,31 +392,34 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           tc_fence_after();
           const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBlockN);
           for (int kb = 0; kb < sp.KB; ++kb) {
-            if (!mbar_wait_bounded(full_bar(stage), phase, p.wait_ns)) {
+            if (!mbar_wait_bounded(fb, phase, p.wait_ns)) {
               latch_error(p.err, kErrWaitMmaFull);
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint64_t adesc = smem_desc_k_sw128(smem_u32(sA + stage * kATiles * kTileBytes));
-            const uint64_t bdesc = smem_desc_k_sw128(smem_u32(sB + stage * kTileBytes));
             // 32 B of K per instruction (16 bf16 or 32 E4M3): +2 in the
             // descriptor's 16-byte address field, inside the swizzled rows
 #pragma unroll
             for (int k32 = 0; k32 < 4; ++k32) {
               const uint32_t acc_flag = (kb > 0 || k32 > 0) ? 1u : 0u;
-              if (kFp8) {
-                constexpr uint64_t kTileDesc = kTileBytes >> 4;  // next A tile: h2
-                tc_mma_e4m3_pair(d_tmem, adesc + 2u * k32, bdesc + 2u * k32, idesc, acc_flag);
-                tc_mma_e4m3_pair(d_tmem, adesc + kTileDesc + 2u * k32, bdesc + 2u * k32, idesc, 1u);
-              } else {
-                tc_mma_bf16_pair(d_tmem, adesc + 2u * k32, bdesc + 2u * k32, idesc, acc_flag);
-              }
+              tc_mma_pair_lohi<kFp8>(d_tmem, a_lo + 2u * k32, a_hi, b_lo + 2u * k32, b_hi, idesc, acc_flag);
+              if (kFp8)  // h2 . q^T: the second A tile of the stage
+                tc_mma_pair_lohi<kFp8>(d_tmem, a_lo + (kTileBytes >> 4) + 2u * k32, a_hi, b_lo + 2u * k32, b_hi,
+                                       idesc, 1u);
             }
-            tc_commit_pair_mc(empty_bar(stage), 0x3);  // frees the stage in both CTAs
+            tc_commit_pair_mc(eb, 0x3);  // frees the stage in both CTAs
+            a_lo += kAStep;
+            b_lo += kBStep;
+            fb += 8;
+            eb += 8;
             if (++stage == kStages) {
               stage = 0;
               phase ^= 1u;
+              a_lo = a_lo0;
+              b_lo = b_lo0;
+              fb = full0;
+              eb = empty0;
             }
           }
           if (ok) tc_commit_pair_mc(tfull_bar(acc), 0x3);
@@ -414,8 +428,8 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
-    const int cg = warp >> 2;      // 64-column group of the tile
+    const int quarter = warp & 3;               // TMEM lanes 32*quarter .. +31
+    const int cg = (warp - kEpiWarp0) >> 2;     // 64-column group of the tile
     const int rloc = quarter * 32 + lane;
     // Every epilogue warp runs the same units and named barriers even after
     // a failed wait (it then skips the work), so the barriers cannot deadlock.
