@@ -36,6 +36,10 @@ constexpr int kPartialFields = 7;                 // m2, S, T2, zmax, zarg, gkey
 constexpr int kPartSmemBytes = kColGroups * kBlockM * kPartialFields * 4;
 // best screening key seen so far by each column group, per row of the CTA
 constexpr int kRecSmemBytes = kColGroups * kBlockM * 4;
+// Largest Philox word of each group of 8 logits for the 32 rows of the MMA
+// warp's lane quarter, one tile ahead, computed by the other epilogue warps:
+// [2 buffers][32 rows][kBlockN / 8 groups].
+constexpr int kWmaxSmemBytes = 2 * 32 * (kBlockN / 8) * 4;
 
 // Pipeline of the two head variants.  bf16 embedder: a stage holds one h
 // tile and one E tile of 64 K.  E4M3 embedder: a stage holds the two E4M3
@@ -46,7 +50,8 @@ struct HeadCfg {
   static constexpr int kBlockKElems = kFp8 ? kBlockKFp8 : kBlockK;
   static constexpr int kATiles = kFp8 ? 2 : 1;
   static constexpr int kStageBytes = (kATiles + 1) * kTileBytes;
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256 + kPartSmemBytes + kRecSmemBytes;
+  static constexpr int kSmemBytes =
+      kStages * kStageBytes + 1024 + 256 + kPartSmemBytes + kRecSmemBytes + kWmaxSmemBytes;
 };
 static_assert(HeadCfg<false>::kSmemBytes <= 232448, "bf16 head exceeds 227 KB of shared memory");
 static_assert(HeadCfg<true>::kSmemBytes <= 232448, "FP8 head exceeds 227 KB of shared memory");

@@ -108,12 +108,28 @@ DG_DEV void top2(float& a1, float& a2, float b1, float b2) {
   a1 = hi;
 }
 
+// The Philox words of the 8 consecutive vocabulary entries 4 cb .. 4 cb + 7.
+DG_DEV void philox_words8(uint32_t cb, uint32_t ctr1, uint32_t ctr2, uint32_t ctr3, const uint32_t (&rk0)[10],
+                          const uint32_t (&rk1)[10], uint32_t (&w)[8]) {
+  uint32_t wa[4], wb[4];
+  philox4x32_10_keys(cb, ctr1, ctr2, ctr3, rk0, rk1, wa);
+  philox4x32_10_keys(cb + 1, ctr1, ctr2, ctr3, rk0, rk1, wb);
+#pragma unroll
+  for (int l = 0; l < 4; ++l) {
+    w[l] = wa[l];
+    w[4 + l] = wb[l];
+  }
+}
+
 // Eight consecutive logits of one row: z[0..7] are vocabulary v0 .. v0+7.
 // thr: the best screening key any column group of this row has reached in
 // the current unit (a lower bound on the row's winning key, up to eps).
+// wm_pre: when have_wm (warp-uniform), the group's largest Philox word,
+// computed beforehand by another warp; the words themselves are then drawn
+// here only if the group passes its bound.
 DG_DEV void process8(const float (&z)[8], int v0, float inv_tau, float c2, uint32_t ctr1,
                      uint32_t ctr2, uint32_t ctr3, const uint32_t (&rk0)[10], const uint32_t (&rk1)[10],
-                     float thr, Partial& pt, Screen& sc) {
+                     float thr, bool have_wm, uint32_t wm_pre, Partial& pt, Screen& sc) {
   // ---- group max, argmax of z (ties to the lower index; groups arrive in
   // increasing v)
   const float m01 = fmaxf(z[0], z[1]), m23 = fmaxf(z[2], z[3]);
@@ -167,17 +183,11 @@ DG_DEV void process8(const float (&z)[8], int v0, float inv_tau, float c2, uint3
   if (x0max + (kGumbelMaxNoise + 1e-3f - kGumbelC0) < lim_eps) return;
   const uint32_t cb = static_cast<uint32_t>(v0) >> 2;
   uint32_t w[8];
-  {
-    uint32_t wa[4], wb[4];
-    philox4x32_10_keys(cb, ctr1, ctr2, ctr3, rk0, rk1, wa);
-    philox4x32_10_keys(cb + 1, ctr1, ctr2, ctr3, rk0, rk1, wb);
-#pragma unroll
-    for (int l = 0; l < 4; ++l) {
-      w[l] = wa[l];
-      w[4 + l] = wb[l];
-    }
-  }
-  {
+  if (have_wm) {
+    if (__fmaf_rn(lg2_exp1_approx(wm_pre), -kLn2, x0max) < lim_eps) return;
+    philox_words8(cb, ctr1, ctr2, ctr3, rk0, rk1, w);
+  } else {
+    philox_words8(cb, ctr1, ctr2, ctr3, rk0, rk1, w);
     const uint32_t wm = max(max(max(w[0], w[1]), max(w[2], w[3])), max(max(w[4], w[5]), max(w[6], w[7])));
     if (__fmaf_rn(lg2_exp1_approx(wm), -kLn2, x0max) < lim_eps) return;
   }
@@ -223,8 +233,8 @@ DG_DEV void process8(const float (&z)[8], int v0, float inv_tau, float c2, uint3
 // logits dump, then the group's reductions.
 template <bool kFp8>
 DG_DEV void epi_group(const uint32_t* r, int v0, int row, float rinv, float inv_tau, float c2,
-                      uint32_t ctr1, uint32_t ctr2, uint32_t ctr3, float thr, const HeadParams& p, Partial& pt,
-                      Screen& sc) {
+                      uint32_t ctr1, uint32_t ctr2, uint32_t ctr3, float thr, bool have_wm, uint32_t wm_pre,
+                      const HeadParams& p, Partial& pt, Screen& sc) {
   float z[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) z[j] = __uint_as_float(r[j]);
@@ -240,7 +250,7 @@ DG_DEV void epi_group(const uint32_t* r, int v0, int row, float rinv, float inv_
     dst[0] = make_float4(z[0], z[1], z[2], z[3]);
     dst[1] = make_float4(z[4], z[5], z[6], z[7]);
   }
-  process8(z, v0, inv_tau, c2, ctr1, ctr2, ctr3, p.rk0, p.rk1, thr, pt, sc);
+  process8(z, v0, inv_tau, c2, ctr1, ctr2, ctr3, p.rk0, p.rk1, thr, have_wm, wm_pre, pt, sc);
 }
 
 // Named barrier over the epilogue warps only (barrier 1).
@@ -263,13 +273,15 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   uint8_t* sA = smem;
   uint8_t* sB = smem + kStages * kATiles * kTileBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sB + kStages * kTileBytes);
-  // barriers: full[S], empty[S], tfull[2], tempty[2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 4);
+  // barriers: full[S], empty[S], tfull[2], tempty[2], wfull[2], wempty[2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 8);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   // [column group][field][row of the CTA half]
   float* sPart = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);
   // [column group][row of the CTA half]: best screening key of the unit so far
   volatile float* sRec = sPart + kColGroups * kPartialFields * kBlockM;
+  // [buffer][group of 8 columns][row of the MMA warp's lane quarter]
+  uint32_t* sWmax = reinterpret_cast<uint32_t*>(sPart + kColGroups * kPartialFields * kBlockM + kColGroups * kBlockM);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -282,6 +294,8 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   auto empty_bar = [&](int s) { return smem_u32(&bars[kStages + s]); };
   auto tfull_bar = [&](int a) { return smem_u32(&bars[2 * kStages + a]); };
   auto tempty_bar = [&](int a) { return smem_u32(&bars[2 * kStages + 2 + a]); };
+  auto wfull_bar = [&](int b) { return smem_u32(&bars[2 * kStages + 4 + b]); };
+  auto wempty_bar = [&](int b) { return smem_u32(&bars[2 * kStages + 6 + b]); };
 
   if (threadIdx.x == 0) {
     prefetch_tensormap(&tmA);
@@ -294,6 +308,8 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1);               // one multicast commit per tile
       mbar_init(tempty_bar(a), 2 * kEpiWarps);  // every epilogue warp of the pair
+      mbar_init(wfull_bar(a), kEpiWarps - 4);   // the 12 word-helper warps
+      mbar_init(wempty_bar(a), 4);              // the MMA quarter's 4 warps
     }
     *s_abort = 0;
     fence_mbarrier_init();
@@ -431,10 +447,48 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     const int quarter = warp & 3;               // TMEM lanes 32*quarter .. +31
     const int cg = (warp - kEpiWarp0) >> 2;     // 64-column group of the tile
     const int rloc = quarter * 32 + lane;
+    // Integer multiplies next to the MMA issuer slow the tensor core, so the
+    // Philox words that bound each group of 8 logits of the MMA warp's lane
+    // quarter are drawn one tile ahead by the other 12 epilogue warps
+    // (helpers) into sWmax; the MMA quarter's warps draw words themselves
+    // only for the rare groups that pass their bound.
+    constexpr int kMmaQuarter = kMmaWarp & 3;
+    constexpr int kTileGroups = kBlockN / 8;  // 32 groups of 8 columns per tile
+    const bool mma_quarter = quarter == kMmaQuarter;
+    const int hidx = cg * 3 + (quarter > kMmaQuarter ? quarter - 1 : quarter);  // helpers: 0..11
+    // Helpers: the largest Philox word of every group of tile t (row tile m_t,
+    // vocabulary tile n_t) for the MMA quarter's 32 rows, into buffer t & 1.
+    auto produce_words = [&](int t, int m_t, int n_t) -> bool {
+      const int buf = t & 1;
+      if (!mbar_wait_bounded(wempty_bar(buf), ((t >> 1) & 1) ^ 1u, p.wait_ns)) {
+        latch_error(p.err, kErrWaitEpilogue);
+        *s_abort = 1;
+        return false;
+      }
+      uint32_t* dst = sWmax + buf * (kTileGroups * 32);
+      for (int i = hidx * 32 + lane; i < kTileGroups * 32; i += (kEpiWarps - 4) * 32) {
+        const int r = i & 31, g = i >> 5;
+        const int hrow = m_t * kPairM + static_cast<int>(rank) * kBlockM + kMmaQuarter * 32 + r;
+        const int hb = hrow >> 8;
+        uint32_t w[8];
+        philox_words8(static_cast<uint32_t>(n_t * kBlockN + g * 8) >> 2,
+                      static_cast<uint32_t>(hrow & 255) | (kPurposeGumbel << 16), static_cast<uint32_t>(p.cp[hb].k),
+                      static_cast<uint32_t>(hb), p.rk0, p.rk1, w);
+        dst[g * 32 + r] = max(max(max(w[0], w[1]), max(w[2], w[3])), max(max(w[4], w[5]), max(w[6], w[7])));
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(wfull_bar(buf));
+      return true;
+    };
     // Every epilogue warp runs the same units and named barriers even after
     // a failed wait (it then skips the work), so the barriers cannot deadlock.
     int tile = 0;
     bool ok = true;
+    if (!mma_quarter) {
+      int m, n0, n1, q;
+      unit_range(sp, pair, m, n0, n1, q);
+      ok = produce_words(0, m, n0);
+    }
     for (int u = pair; u < sp.units; u += npairs) {
       int m, n0, n1, q;
       unit_range(sp, u, m, n0, n1, q);
@@ -459,6 +513,26 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         const uint32_t acc_phase = (tile >> 1) & 1;
         if (ok && *s_abort) ok = false;
         if (!ok) continue;
+        if (!mma_quarter) {
+          // the words of the next tile (this unit's next, or the next unit's first)
+          int mn = m, nn = n + 1;
+          bool more = nn < n1;
+          if (!more && u + npairs < sp.units) {
+            int n1n, qn;
+            unit_range(sp, u + npairs, mn, nn, n1n, qn);
+            more = true;
+          }
+          if (more && !produce_words(tile + 1, mn, nn)) {
+            ok = false;
+            continue;
+          }
+        } else if (!mbar_wait_bounded(wfull_bar(tile & 1), (tile >> 1) & 1, p.wait_ns)) {
+          latch_error(p.err, kErrWaitEpilogue);
+          *s_abort = 1;
+          ok = false;
+          continue;
+        }
+        const uint32_t* wsrc = sWmax + (tile & 1) * (kTileGroups * 32) + cg * 8 * 32 + lane;
         if (!mbar_wait_bounded(tfull_bar(acc), acc_phase, p.wait_ns)) {
           latch_error(p.err, kErrWaitEpilogue);
           *s_abort = 1;
@@ -486,10 +560,12 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 #pragma unroll 1
         for (int g = 0; g < kGroups; g += 2) {
           tmem_load8_issue(tbase + 8 * (g + 1), rb);
-          epi_group<kFp8>(ra, vbase + 8 * g, row, rinv, inv_tau, c2, ctr1, ctr2, ctr3, thr, p, pt, sc);
+          epi_group<kFp8>(ra, vbase + 8 * g, row, rinv, inv_tau, c2, ctr1, ctr2, ctr3, thr, mma_quarter,
+                          mma_quarter ? wsrc[g * 32] : 0u, p, pt, sc);
           tmem_load8_wait(rb);
           if (g + 2 < kGroups) tmem_load8_issue(tbase + 8 * (g + 2), ra);
-          epi_group<kFp8>(rb, vbase + 8 * (g + 1), row, rinv, inv_tau, c2, ctr1, ctr2, ctr3, thr, p, pt, sc);
+          epi_group<kFp8>(rb, vbase + 8 * (g + 1), row, rinv, inv_tau, c2, ctr1, ctr2, ctr3, thr, mma_quarter,
+                          mma_quarter ? wsrc[(g + 1) * 32] : 0u, p, pt, sc);
           tmem_load8_wait(ra);
           __syncwarp();
         }
@@ -505,6 +581,7 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             mbar_arrive(tempty_bar(acc));
           else
             mbar_arrive_remote(mapa_shared(tempty_bar(acc), 0));
+          if (mma_quarter) mbar_arrive(wempty_bar(tile & 1));  // its words are consumed
         }
       }
       if (ok) screen_flush(sc, pt, inv_tau);
