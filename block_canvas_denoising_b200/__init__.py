@@ -16,7 +16,8 @@ import numpy as np
 
 __all__ = ["DGError", "Params", "lib", "workspace_size", "Workspace", "denoise_step",
            "debug_logits", "device_status", "denoise_loop", "debug_gumbel",
-           "selftest_bounded_wait", "set_head_events", "denoise_step_noalloc", "STATUS", "E_BF16", "E_FP8_E4M3"]
+           "selftest_bounded_wait", "set_head_events", "denoise_step_noalloc", "STATUS", "E_BF16", "E_FP8_E4M3",
+           "SELECT_CUMSUM", "SELECT_MI", "SELECT_TOPK"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdg.so")
@@ -43,7 +44,12 @@ class _Shape(ctypes.Structure):
 class _Params(ctypes.Structure):
     _fields_ = [("tau0", ctypes.c_double), ("tau1", ctypes.c_double), ("max_steps", ctypes.c_int32),
                 ("entropy_bound", ctypes.c_double), ("stop_entropy", ctypes.c_double),
-                ("seed", ctypes.c_uint64)]
+                ("seed", ctypes.c_uint64), ("selection_rule", ctypes.c_int32), ("top_k", ctypes.c_int32)]
+
+
+SELECT_CUMSUM = 0
+SELECT_MI = 1
+SELECT_TOPK = 2
 
 
 _HIDDEN_FN = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
@@ -59,10 +65,13 @@ class Params:
     entropy_bound: float = 0.1
     stop_entropy: float = 0.005
     seed: int = 1234
+    selection_rule: int = SELECT_CUMSUM
+    top_k: int = 1
 
     def c(self) -> _Params:
         return _Params(self.tau0, self.tau1, self.max_steps, self.entropy_bound,
-                       self.stop_entropy, int(self.seed) & 0xFFFFFFFFFFFFFFFF)
+                       self.stop_entropy, int(self.seed) & 0xFFFFFFFFFFFFFFFF,
+                       int(self.selection_rule), int(self.top_k))
 
 
 _lib = None

@@ -71,6 +71,8 @@ dg_status check_params(const dg_params* p) {
   if (p->max_steps < 1 || !finite_pos(p->tau0) || !finite_pos(p->tau1)) return DG_ERR_INVALID_ARG;
   if (!(p->entropy_bound >= 0.0 && p->entropy_bound < 1e300)) return DG_ERR_INVALID_ARG;
   if (!(p->stop_entropy >= 0.0 && p->stop_entropy < 1e300)) return DG_ERR_INVALID_ARG;
+  if (p->selection_rule < DG_SELECT_CUMSUM || p->selection_rule > DG_SELECT_TOPK) return DG_ERR_INVALID_ARG;
+  if (p->selection_rule == DG_SELECT_TOPK && (p->top_k < 1 || p->top_k > 256)) return DG_ERR_INVALID_ARG;
   return DG_OK;
 }
 
@@ -241,6 +243,8 @@ dg_status run_step(const StepArgs& a) {
   mp.seed_lo = hp.seed_lo;
   mp.seed_hi = hp.seed_hi;
   mp.entropy_bound = pr.entropy_bound;
+  mp.selection_rule = pr.selection_rule;
+  mp.top_k = pr.top_k;
   mp.stop_entropy = pr.stop_entropy;
   memcpy(mp.cp, cps, sizeof(cps));
   if (!cuda_ok(launch_merge(mp, a.stream), "merge kernel launch")) return DG_ERR_CUDA;
@@ -286,6 +290,8 @@ dg_params dg_default_params(void) {
   p.entropy_bound = 0.1;
   p.stop_entropy = 0.005;
   p.seed = 1234;
+  p.selection_rule = DG_SELECT_CUMSUM;
+  p.top_k = 1;
   return p;
 }
 

@@ -104,6 +104,8 @@ struct MergeParams {
   uint32_t seed_lo, seed_hi;
   double entropy_bound;
   double stop_entropy;
+  int32_t selection_rule;  // dg_selection
+  int32_t top_k;
   CanvasParam cp[DG_MAX_B];
 };
 

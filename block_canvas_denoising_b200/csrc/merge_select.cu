@@ -8,7 +8,9 @@
 //   * selection ([Docs] "DiffusionGemma", Recommended serving configuration,
 //     token selection, entropy bound 0.1): slots ordered by (entropy, slot);
 //     slot s is accepted when the running entropy sum up to and including s
-//     is <= the bound, and the lowest-entropy slot always is;
+//     is <= the bound, and the lowest-entropy slot always is (the default
+//     rule); the variants accept when the sum over the slots before s is
+//     <= the bound, or when s is among the top_k lowest;
 //   * renoise (same row: unselected tokens fully renoised; [Report]
 //     "DiffusionGemma Technical Report", Figure 3: uniform noise): token
 //     (r V) >> 32 from Philox counter (0, slot | 1 << 16, k, b), lane 0;
@@ -118,21 +120,29 @@ merge_select_kernel(const __grid_constant__ MergeParams p) {
   s_key[s] = key;
   s_h[s] = H;
   __syncthreads();
-  // four independent running sums over i = j mod 4, added in a fixed order
+  // Running sums over the slots ordered before this one (exclusive) or up
+  // to and including it (inclusive): four independent float64 sums over
+  // i = j mod 4, added in a fixed order.  The rank is the slot's position.
   double cs[4] = {0.0, 0.0, 0.0, 0.0};
   int rk[4] = {0, 0, 0, 0};
+  const bool inclusive = p.selection_rule == DG_SELECT_CUMSUM;
 #pragma unroll 4
   for (int i = 0; i < 256; i += 4) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const unsigned long long ki = s_key[i + j];
-      if (ki <= key) cs[j] += static_cast<double>(s_h[i + j]);
-      rk[j] += (ki < key) ? 1 : 0;
+      const bool before = ki < key;
+      if (before || (inclusive && ki == key)) cs[j] += static_cast<double>(s_h[i + j]);
+      rk[j] += before ? 1 : 0;
     }
   }
   const double csum = (cs[0] + cs[1]) + (cs[2] + cs[3]);
   const int rank = (rk[0] + rk[1]) + (rk[2] + rk[3]);
-  const bool accepted = (csum <= p.entropy_bound) || (rank == 0);
+  bool accepted;
+  if (p.selection_rule == DG_SELECT_TOPK)
+    accepted = rank < p.top_k;
+  else  // CUMSUM: inclusive sum <= bound, at least one; MI: exclusive sum <= bound
+    accepted = (csum <= p.entropy_bound) || (rank == 0);
 
   // ---- renoise
   int tok = samp;

@@ -73,15 +73,30 @@ typedef struct {
 
 #define DG_MAX_B 256
 
+/* Selection rule: which prefix of the slots ordered by (entropy, slot) is
+ * accepted each step.  Every rule accepts at least one slot.
+ *   DG_SELECT_CUMSUM  the longest prefix whose entropy sum is <= entropy_bound
+ *                     (default; this library's reading of the [Docs]
+ *                     token-selection row, which bounds a mutual-information
+ *                     estimate by 0.1 and gives no formula).
+ *   DG_SELECT_MI      the longest prefix whose entropy sum minus its largest
+ *                     entropy is <= entropy_bound (the usual form of such a
+ *                     bound in the literature; not stated on the pages).
+ *   DG_SELECT_TOPK    the top_k lowest-entropy slots (1 <= top_k <= L). */
+typedef enum { DG_SELECT_CUMSUM = 0, DG_SELECT_MI = 1, DG_SELECT_TOPK = 2 } dg_selection;
+
 /* Sampler parameters; dg_default_params() gives the [Docs] serving
- * defaults (tau0 0.8, tau1 0.4, 48 steps, bound 0.1, stop 0.005). */
+ * defaults (tau0 0.8, tau1 0.4, 48 steps, bound 0.1, stop 0.005,
+ * DG_SELECT_CUMSUM). */
 typedef struct {
-  double tau0;           /* temperature at step 0 */
-  double tau1;           /* temperature at step max_steps-1 */
-  int32_t max_steps;     /* N, at most this many steps per canvas */
-  double entropy_bound;  /* selection bound on the cumulative entropy */
-  double stop_entropy;   /* adaptive stop: canvas-mean entropy threshold */
-  uint64_t seed;         /* Philox4x32-10 key (low word, high word) */
+  double tau0;             /* temperature at step 0 */
+  double tau1;             /* temperature at step max_steps-1 */
+  int32_t max_steps;       /* N, at most this many steps per canvas */
+  double entropy_bound;    /* selection bound on the entropies (see dg_selection) */
+  double stop_entropy;     /* adaptive stop: canvas-mean entropy threshold */
+  uint64_t seed;           /* Philox4x32-10 key (low word, high word) */
+  int32_t selection_rule;  /* a dg_selection */
+  int32_t top_k;           /* slots accepted by DG_SELECT_TOPK */
 } dg_params;
 
 dg_params dg_default_params(void);

@@ -53,7 +53,7 @@ def replay_step(z32, *, B: int, L: int, step_idx, has_prev, prev_argmax,
         if entropy_in is not None:
             H = np.asarray(entropy_in[i * L:(i + 1) * L], dtype=np.float64)
         amax = argmax_lowest(zc)
-        acc, _, om = select(H, params.entropy_bound)
+        acc, _, om = select(H, params.entropy_bound, params.selection_rule, params.top_k)
         noise = renoise_tokens(b, k, L, V, params.seed)
         canvas = np.where(acc == 1, samp, noise).astype(np.int32)
         st, _ = stop_flag(H, amax, prev_argmax[b * L:(b + 1) * L], bool(has_prev[b]),

@@ -40,6 +40,12 @@ PURPOSE_GUMBEL = 0
 PURPOSE_RENOISE = 1
 
 
+# selection rules (the default is this project's reading of the pages)
+SELECT_CUMSUM = 0   # longest sorted prefix with sum of entropies <= bound, at least one
+SELECT_MI = 1       # longest sorted prefix with sum minus its largest entropy <= bound
+SELECT_TOPK = 2     # the top_k lowest-entropy slots
+
+
 @dataclass
 class Params:
     tau0: float = TAU0
@@ -48,6 +54,8 @@ class Params:
     entropy_bound: float = ENTROPY_BOUND
     stop_entropy: float = STOP_ENTROPY
     seed: int = 1234
+    selection_rule: int = SELECT_CUMSUM
+    top_k: int = 1
 
 
 # --------------------------------------------------------------------------
@@ -212,28 +220,54 @@ def gumbel_sample(x: np.ndarray, words: np.ndarray):
 # a7: entropy-bounded selection, a8: renoise, a9: stop
 # --------------------------------------------------------------------------
 
-def select(H: np.ndarray, bound: float = ENTROPY_BOUND):
+def select(H: np.ndarray, bound: float = ENTROPY_BOUND, rule: int = SELECT_CUMSUM, top_k: int = 1):
     """Entropy-bounded acceptance of one canvas.
 
-    Sort the slots by entropy (ties to the lower slot), take the inclusive
-    running sum c_j, accept the first n = max(1, #{j : c_j <= bound}).
-    [Docs] token-selection row: the lowest-entropy tokens are chosen so that
-    the bound holds; the cumulative-sum form is this project's reading of
-    that mutual-information bound.  Returns (accept uint8, n, margin) where
-    margin is the closest call at the cut.
+    Sort the slots by entropy (ties to the lower slot) and accept a prefix of
+    that order:
+      * SELECT_CUMSUM (default): with the inclusive running sum c_j, the first
+        n = max(1, #{j : c_j <= bound}).  [Docs] token-selection row: the
+        lowest-entropy tokens are chosen so that the bound holds; the
+        cumulative-sum form is this project's reading of that
+        mutual-information bound.
+      * SELECT_MI: the longest prefix whose entropy sum minus its largest
+        entropy is <= bound, i.e. with the exclusive running sum e_j (the sum
+        over the slots ranked before j; e_0 = 0), n = #{j : e_j <= bound} >= 1.
+        A bound of this shape is the usual form in the literature on
+        entropy-bounded samplers; the pages do not state it.
+      * SELECT_TOPK: the top_k lowest-entropy slots.
+    Returns (accept uint8, n, margin) where margin is the closest call at the
+    cut (for the sums: distance of the deciding sums from the bound, or the
+    entropy gap at the cut; for top-k: the entropy gap at the cut).
     """
     H = np.asarray(H, dtype=np.float64)
     L = H.shape[0]
     order = np.lexsort((np.arange(L), H))
-    c = np.cumsum(H[order])
-    n = max(1, int(np.count_nonzero(c <= bound)))
+    Hs = H[order]
+    c = np.cumsum(Hs)
+    margins = []
+    if rule == SELECT_CUMSUM:
+        n = max(1, int(np.count_nonzero(c <= bound)))
+        margins.append(abs(c[n - 1] - bound))
+        if n < L:
+            margins.append(abs(c[n] - bound))
+    elif rule == SELECT_MI:
+        e = np.concatenate([[0.0], c[:-1]])
+        n = int(np.count_nonzero(e <= bound))
+        margins.append(abs(e[n - 1] - bound))
+        if n < L:
+            margins.append(abs(e[n] - bound))
+    elif rule == SELECT_TOPK:
+        if not 1 <= top_k <= L:
+            raise ValueError("top_k out of range")
+        n = int(top_k)
+    else:
+        raise ValueError("unknown selection rule")
     acc = np.zeros(L, dtype=np.uint8)
     acc[order[:n]] = 1
-    margins = [abs(c[n - 1] - bound)]
     if n < L:
-        margins.append(abs(c[n] - bound))
-        margins.append(abs(H[order[n]] - H[order[n - 1]]))
-    return acc, n, float(min(margins))
+        margins.append(abs(Hs[n] - Hs[n - 1]))
+    return acc, n, float(min(margins)) if margins else float("inf")
 
 
 def renoise_tokens(b: int, k: int, L: int, V: int, seed: int) -> np.ndarray:
@@ -296,7 +330,7 @@ def denoise_step(h_bits, *, E_bits=None, q=None, s=None, B: int, L: int = 256,
             H[s0:s1] = entropy(x)
             w = gumbel_words(np.arange(s0, s1), b, k, V, params.seed)
             samp[s0:s1], gm[s0:s1] = gumbel_sample(x, w)
-        acc, n, om = select(H, params.entropy_bound)
+        acc, n, om = select(H, params.entropy_bound, params.selection_rule, params.top_k)
         noise = renoise_tokens(b, k, L, V, params.seed)
         canvas = np.where(acc == 1, samp, noise).astype(np.int32)
         st, sm = stop_flag(H, amax, prev_argmax[b * L:(b + 1) * L], bool(has_prev[b]),

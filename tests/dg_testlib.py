@@ -81,7 +81,7 @@ def run_step(h_bits, E_bits, step_idx, has_prev, prev_argmax, canvas0, params, *
 
 def oparams(p) -> OParams:
     return OParams(tau0=p.tau0, tau1=p.tau1, max_steps=p.max_steps, entropy_bound=p.entropy_bound,
-                   stop_entropy=p.stop_entropy, seed=p.seed)
+                   stop_entropy=p.stop_entropy, seed=p.seed, selection_rule=p.selection_rule, top_k=p.top_k)
 
 
 def rows_of(canvases, L=256):

@@ -43,6 +43,26 @@ def test_library_exports_every_declared_symbol(libdg):
 def test_default_params_are_serving_defaults(libdg):
     p = libdg.dg_default_params()
     assert (p.tau0, p.tau1, p.max_steps, p.entropy_bound, p.stop_entropy) == (0.8, 0.4, 48, 0.1, 0.005)
+    # the struct layout of the binding matches the library's (fields after the
+    # seed read back as set by the C side)
+    assert (p.seed, p.selection_rule, p.top_k) == (1234, dg.SELECT_CUMSUM, 1)
+
+
+def test_selection_rule_checks(libdg):
+    # unknown rule, top-k out of [1, 256]: refused on the host
+    def call(rule, k):
+        prm = dg.Params(selection_rule=rule, top_k=k).c()
+        shp = dg._Shape(1, 256, 512, 8192, 0)
+        ks = np.zeros(1, np.int32)
+        hp = np.zeros(1, np.uint8)
+        fake = ctypes.c_void_p(256)
+        return libdg.dg_denoise_step(ctypes.byref(shp), ctypes.byref(prm), fake, fake, None,
+                                     ks.ctypes.data_as(ctypes.c_void_p), hp.ctypes.data_as(ctypes.c_void_p),
+                                     None, *([fake] * 7), fake, ctypes.c_size_t(1 << 30), None)
+    assert call(3, 1) == 1
+    assert call(-1, 1) == 1
+    assert call(dg.SELECT_TOPK, 0) == 1
+    assert call(dg.SELECT_TOPK, 257) == 1
 
 
 def test_error_strings(libdg):

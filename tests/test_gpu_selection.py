@@ -1,0 +1,89 @@
+"""Selection-rule variants and the longer step schedule through the C ABI.
+
+The default rule (cumulative entropy sum within the bound) is covered by the
+other parity files; here the alternatives run on low-entropy canvases (the
+loop's stand-in hidden states at early steps, where the accepted prefix ends
+mid-canvas): the mutual-information-style bound (sum minus the largest
+entropy of the prefix), fixed top-k, and a 192-step temperature schedule.
+Each case is compared with the oracle and replayed bit-exactly on the
+device's logits and entropies.
+"""
+import numpy as np
+import pytest
+
+import synth
+from dg_testlib import check_replay, compare_with_oracle, run_step
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import block_canvas_denoising_b200 as dg  # noqa: E402
+from block_canvas_denoising_b200 import build as dg_build  # noqa: E402
+
+dg_build.build()
+L = 256
+
+
+def _low_entropy_case(ks, d=512, V=8192):
+    B = len(ks)
+    E = synth.embedder_normal(V, d, seed=1)
+    y = synth.loop_targets(L, V, seed=3, B=B)
+    h = np.concatenate([synth.loop_hidden(int(k), y, E, seed=4)[b * L:(b + 1) * L] for b, k in enumerate(ks)])
+    canvas0 = synth.canvas_uniform(B, L, V, seed=0)
+    return h, E, canvas0
+
+
+@pytest.mark.parametrize("rule,bound,k,expect_mid", [
+    (dg.SELECT_CUMSUM, 0.1, 1, True),
+    (dg.SELECT_MI, 0.1, 1, True),
+    (dg.SELECT_MI, 0.3, 1, True),
+    (dg.SELECT_TOPK, 0.1, 1, False),
+    (dg.SELECT_TOPK, 0.1, 17, False),
+    (dg.SELECT_TOPK, 0.1, 256, False),
+])
+def test_selection_rules_parity_and_replay(rule, bound, k, expect_mid):
+    # steps 3-5: the accepted prefix ends between slot 1 and slot 60, where
+    # the canvases' neighbouring entropies are at least ~1e-6 apart (step 6
+    # puts the cut among entropies ~1e-7 apart, where float32 and float64
+    # entropies order differently and whole swaps exceed the 0.1 % budget)
+    ks = np.array([3, 4, 5], np.int32)
+    h, E, canvas0 = _low_entropy_case(ks)
+    B = len(ks)
+    hp = np.ones(B, np.uint8)
+    prev = np.zeros(B * L, np.int32)
+    params = dg.Params(selection_rule=rule, entropy_bound=bound, top_k=k)
+    g = run_step(h, E, ks, hp, prev, canvas0, params)
+    compare_with_oracle(g, h, E, ks, hp, prev, params)
+    check_replay(g, ks, hp, prev, params)
+    counts = g["accept"].reshape(B, L).sum(axis=1)
+    if rule == dg.SELECT_TOPK:
+        assert np.all(counts == k)
+    elif expect_mid:
+        assert counts.min() >= 1 and np.any((counts > 1) & (counts < L)), counts
+
+
+def test_mi_rule_accepts_a_superset_of_the_cumsum_rule():
+    ks = np.array([4, 5, 6], np.int32)
+    h, E, canvas0 = _low_entropy_case(ks)
+    hp = np.ones(3, np.uint8)
+    prev = np.zeros(3 * L, np.int32)
+    g_c = run_step(h, E, ks, hp, prev, canvas0, dg.Params(selection_rule=dg.SELECT_CUMSUM), debug=False)
+    g_m = run_step(h, E, ks, hp, prev, canvas0, dg.Params(selection_rule=dg.SELECT_MI), debug=False)
+    assert np.all(g_m["accept"] >= g_c["accept"])
+    assert np.array_equal(g_m["entropy"], g_c["entropy"])
+
+
+@pytest.mark.parametrize("k", [0, 100, 191])
+def test_longer_schedule_192_steps(k):
+    # tau runs from 0.8 at k = 0 to 0.4 at k = N - 1 for any N
+    ks = np.array([k], np.int32)
+    h, E, canvas0 = _low_entropy_case(np.array([4]))
+    hp = np.zeros(1, np.uint8)
+    prev = np.zeros(L, np.int32)
+    params = dg.Params(max_steps=192)
+    g = run_step(h, E, ks, hp, prev, canvas0, params)
+    compare_with_oracle(g, h, E, ks, hp, prev, params)
+    check_replay(g, ks, hp, prev, params)

@@ -313,3 +313,65 @@ def test_replay_of_rounded_logits_agrees_with_f64_draw():
     assert np.all(r64["gumbel_margin"][diff] < 1e-3)
     assert diff.mean() <= 0.01
     assert np.abs(rr["entropy"] - r64["entropy"]).max() < 1e-5
+
+
+# ---- selection-rule variants ------------------------------------------------
+
+def test_select_mi_rule_hand_case():
+    from oracle.step import SELECT_MI, SELECT_CUMSUM
+    H = np.array([0.05, 0.02, 0.03, 0.5, 0.01])
+    # sorted 0.01 (s4), 0.02 (s1), 0.03 (s2), 0.05 (s0), 0.5 (s3); the sum of a
+    # prefix minus its largest entropy is 0, 0.01, 0.03, 0.06, 0.11
+    acc, n, _ = S.select(H, 0.1, SELECT_MI)
+    assert n == 4 and acc.tolist() == [1, 1, 1, 0, 1]
+    acc_c, n_c, _ = S.select(H, 0.1, SELECT_CUMSUM)
+    assert n_c == 3 and acc_c.tolist() == [0, 1, 1, 0, 1]
+
+
+def test_select_mi_rule_brute_force_definition():
+    # longest prefix of the (entropy, slot) order whose sum minus its largest
+    # entropy is <= bound, by plain loops over every prefix
+    from oracle.step import SELECT_MI
+    rng = np.random.default_rng(17)
+    for trial in range(300):
+        L = int(rng.integers(1, 9))
+        H = rng.exponential(0.04, L) * (rng.random(L) < 0.8)
+        bound = float(rng.choice([0.0, 0.01, 0.05, 0.1, 0.3]))
+        order = sorted(range(L), key=lambda i: (H[i], i))
+        best = 0
+        for n in range(1, L + 1):
+            pre = [H[i] for i in order[:n]]
+            if sum(pre) - max(pre) <= bound:
+                best = n
+        want = np.zeros(L, np.uint8)
+        want[order[:best]] = 1
+        acc, n, _ = S.select(H, bound, SELECT_MI)
+        assert n == best and np.array_equal(acc, want), (trial, H, bound)
+
+
+def test_select_mi_contains_cumsum_and_is_monotone():
+    from oracle.step import SELECT_MI, SELECT_CUMSUM
+    rng = np.random.default_rng(5)
+    for _ in range(100):
+        H = rng.exponential(0.02, 256)
+        a_c, _, _ = S.select(H, 0.1, SELECT_CUMSUM)
+        a_m, _, _ = S.select(H, 0.1, SELECT_MI)
+        assert np.all(a_m >= a_c)
+        prev = 0
+        for g in (0.0, 0.02, 0.05, 0.1, 0.2, 1.0):
+            _, n, _ = S.select(H, g, SELECT_MI)
+            assert n >= max(prev, 1)
+            prev = n
+
+
+def test_select_topk_rule():
+    from oracle.step import SELECT_TOPK
+    H = np.array([0.3, 0.1, 0.1, 0.0, 0.2])
+    acc, n, m = S.select(H, 0.1, SELECT_TOPK, 3)
+    assert n == 3 and acc.tolist() == [0, 1, 1, 1, 0]     # ties to the lower slot
+    acc, n, m = S.select(np.zeros(6), 0.1, SELECT_TOPK, 2)
+    assert acc.tolist() == [1, 1, 0, 0, 0, 0] and m == 0.0
+    acc, n, _ = S.select(H, 0.1, SELECT_TOPK, 5)
+    assert acc.sum() == 5
+    with pytest.raises(ValueError):
+        S.select(H, 0.1, SELECT_TOPK, 0)
