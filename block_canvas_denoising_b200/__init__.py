@@ -17,7 +17,8 @@ import numpy as np
 __all__ = ["DGError", "Params", "lib", "workspace_size", "Workspace", "denoise_step",
            "debug_logits", "device_status", "denoise_loop", "debug_gumbel",
            "selftest_bounded_wait", "set_head_events", "denoise_step_noalloc", "STATUS", "E_BF16", "E_FP8_E4M3",
-           "SELECT_CUMSUM", "SELECT_MI", "SELECT_TOPK"]
+           "SELECT_CUMSUM", "SELECT_MI", "SELECT_TOPK", "partials_count", "head_partials", "merge_partials",
+           "gather_partials"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdg.so")
@@ -105,6 +106,14 @@ def lib() -> ctypes.CDLL:
         L.dg_denoise_step_noalloc.argtypes = step_args + [P]
         L.dg_denoise_step_noalloc.restype = ctypes.c_int
         L.dg_last_error_message.restype = ctypes.c_char_p
+        L.dg_partials_count.restype = ctypes.c_int32
+        L.dg_partials_count.argtypes = [ctypes.POINTER(_Shape)]
+        L.dg_head_partials.restype = ctypes.c_int
+        L.dg_head_partials.argtypes = [ctypes.POINTER(_Shape), ctypes.POINTER(_Params), ctypes.c_int32,
+                                       P, P, P, P, P, P, ctypes.c_size_t, P]
+        L.dg_merge_partials.restype = ctypes.c_int
+        L.dg_merge_partials.argtypes = [ctypes.POINTER(_Shape), ctypes.POINTER(_Params), P, ctypes.c_int32,
+                                        ctypes.c_int32, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         for name in ("dg_workspace_init", "dg_denoise_step", "dg_debug_logits", "dg_device_status",
                      "dg_denoise_loop", "dg_selftest_bounded_wait", "dg_debug_gumbel",
                      "dg_set_head_events"):
@@ -295,3 +304,60 @@ def selftest_bounded_wait(limit_ns: int, ws: Workspace, stream=None) -> int:
     """Run the bounded-wait self test; returns the status code (6 = timed out as designed)."""
     return int(lib().dg_selftest_bounded_wait(ctypes.c_uint64(limit_ns), _ptr(ws.buf),
                                               ctypes.c_size_t(ws.nbytes), _stream(stream)))
+
+
+# ---------------------------------------------------------------------------
+# vocabulary-sharded step (dg_head_partials / dg_merge_partials)
+# ---------------------------------------------------------------------------
+
+def partials_count(B: int, d: int, V_shard: int, e_dtype: int = E_BF16, L: int = 256) -> int:
+    """Records per row that one shard's head writes (``dg_partials_count``)."""
+    return int(lib().dg_partials_count(ctypes.byref(_shape(B, d, V_shard, e_dtype, L))))
+
+
+def head_partials(h, E_shard, v_offset: int, step_idx, partials, ws: Workspace, params: Params = Params(),
+                  e_scale=None, stream=None) -> None:
+    """Head and sampler over vocabulary rows v_offset .. v_offset + len(E_shard) - 1,
+    writing the float32 records [7, B*256, count] into ``partials``."""
+    B = int(len(step_idx))
+    R, d = h.shape
+    shp = _shape(B, d, E_shard.shape[0], E_BF16 if e_scale is None else E_FP8_E4M3, L=R // max(B, 1))
+    prm = params.c()
+    ks = _host(step_idx, np.int32)
+    _check(lib().dg_head_partials(ctypes.byref(shp), ctypes.byref(prm), ctypes.c_int32(v_offset), _ptr(h),
+                                  _ptr(E_shard), _ptr(e_scale), ks.ctypes.data_as(ctypes.c_void_p),
+                                  _ptr(partials), _ptr(ws.buf), ctypes.c_size_t(ws.nbytes), _stream(stream)),
+           "dg_head_partials")
+
+
+def merge_partials(partials, V: int, d: int, step_idx, has_prev, canvas, prev_argmax, accept, entropy, sampled,
+                   argmax, stop, ws: Workspace, params: Params = Params(), active=None, stream=None) -> None:
+    """Merge the gathered records ``partials`` [S, 7, B*256, count] over the
+    whole vocabulary V, then selection, renoise and stop."""
+    B = int(len(step_idx))
+    S, _, R, count = partials.shape
+    shp = _shape(B, d, V, E_BF16, L=R // max(B, 1))
+    prm = params.c()
+    ks = _host(step_idx, np.int32)
+    hp = _host(has_prev, np.uint8)
+    act = None if active is None else _host(active, np.uint8)
+    _check(lib().dg_merge_partials(ctypes.byref(shp), ctypes.byref(prm), _ptr(partials), ctypes.c_int32(S),
+                                   ctypes.c_int32(count), ks.ctypes.data_as(ctypes.c_void_p),
+                                   hp.ctypes.data_as(ctypes.c_void_p),
+                                   None if act is None else act.ctypes.data_as(ctypes.c_void_p),
+                                   _ptr(canvas), _ptr(prev_argmax), _ptr(accept), _ptr(entropy), _ptr(sampled),
+                                   _ptr(argmax), _ptr(stop), _ptr(ws.buf), ctypes.c_size_t(ws.nbytes),
+                                   _stream(stream)), "dg_merge_partials")
+
+
+def gather_partials(local, group=None):
+    """All-gather one rank's records [7, R, count] into [world, 7, R, count]
+    (torch.distributed over the default or given process group; NCCL for
+    CUDA tensors).  The only collective of the sharded step."""
+    import torch
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    local = local.contiguous()
+    out = torch.empty((world * local.shape[0],) + tuple(local.shape[1:]), dtype=local.dtype, device=local.device)
+    dist.all_gather_into_tensor(out, local, group=group)
+    return out.view((world,) + tuple(local.shape))

@@ -107,6 +107,8 @@ bool encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t esize, CUte
   return r == CUDA_SUCCESS;
 }
 
+enum class StepMode { kFull, kHeadOnly, kMergeOnly };
+
 struct StepArgs {
   const dg_shape* shape;
   const dg_params* params;
@@ -127,6 +129,11 @@ struct StepArgs {
   void* workspace;
   size_t ws_bytes;
   cudaStream_t stream;
+  StepMode mode = StepMode::kFull;
+  int32_t v_off = 0;              // head: vocabulary index of E's first row
+  float* part_out = nullptr;      // head only: the records [7][R][P] go here
+  const float* part_in = nullptr; // merge only: S shards' records [S][7][R][P]
+  int32_t S = 1, P = 0;           // merge only
 };
 
 dg_status run_step(const StepArgs& a) {
@@ -135,14 +142,22 @@ dg_status run_step(const StepArgs& a) {
   if ((st = check_params(a.params)) != DG_OK) return st;
   const dg_shape& s = *a.shape;
   const dg_params& pr = *a.params;
-  if (!a.h || !a.E || !a.step_idx || !a.has_prev || !a.canvas || !a.prev_argmax || !a.accept ||
-      !a.entropy || !a.sampled || !a.argmax || !a.stop || !a.workspace)
+  const bool head = a.mode != StepMode::kMergeOnly;
+  const bool merge = a.mode != StepMode::kHeadOnly;
+  if (!a.step_idx || !a.workspace || !aligned16(a.workspace)) return DG_ERR_INVALID_ARG;
+  if (head && (!a.h || !a.E || !aligned16(a.h) || !aligned16(a.E))) return DG_ERR_INVALID_ARG;
+  if (merge && (!a.has_prev || !a.canvas || !a.prev_argmax || !a.accept || !a.entropy || !a.sampled ||
+                !a.argmax || !a.stop))
     return DG_ERR_INVALID_ARG;
-  if (!aligned16(a.h) || !aligned16(a.E) || !aligned16(a.workspace)) return DG_ERR_INVALID_ARG;
   const bool fp8 = s.e_dtype == DG_E_FP8_E4M3;
   // the per-row scale belongs to the FP8 embedder only
-  if (fp8 ? (a.e_scale == nullptr || !aligned16(a.e_scale)) : a.e_scale != nullptr) return DG_ERR_INVALID_ARG;
+  if (head && (fp8 ? (a.e_scale == nullptr || !aligned16(a.e_scale)) : a.e_scale != nullptr))
+    return DG_ERR_INVALID_ARG;
   if (a.logits != nullptr && !aligned16(a.logits)) return DG_ERR_INVALID_ARG;
+  if (a.mode == StepMode::kHeadOnly && (a.part_out == nullptr || !aligned16(a.part_out) || a.v_off < 0 ||
+                                        a.v_off % kBlockN != 0))
+    return DG_ERR_INVALID_ARG;
+  if (a.mode == StepMode::kMergeOnly && (a.part_in == nullptr || a.S < 1 || a.P < 1)) return DG_ERR_INVALID_ARG;
   for (int b = 0; b < s.B; ++b)
     if (a.step_idx[b] < 0 || a.step_idx[b] >= pr.max_steps) return DG_ERR_RANGE;
   if (device_sms() <= 0) return DG_ERR_NO_DEVICE;
@@ -152,85 +167,102 @@ dg_status run_step(const StepArgs& a) {
     return DG_ERR_CUDA;
   }
   const WsLayout ws = ws_layout(s, pairs);
-  if (a.ws_bytes < ws.total) return DG_ERR_WORKSPACE;
+  if (a.ws_bytes < (head ? ws.total : ws.zero_prefix)) return DG_ERR_WORKSPACE;
 
   const int R = s.B * s.L;
   uint8_t* wsb = static_cast<uint8_t*>(a.workspace);
+  uint32_t* row_rec = reinterpret_cast<uint32_t*>(wsb + ws.rec_off);
 
   CanvasParam cps[DG_MAX_B];
   memset(cps, 0, sizeof(cps));
   for (int b = 0; b < s.B; ++b) {
     cps[b].k = a.step_idx[b];
     cps[b].inv_tau = inv_tau_of(pr, a.step_idx[b]);
-    cps[b].has_prev = a.has_prev[b] ? 1 : 0;
+    cps[b].has_prev = (merge && a.has_prev[b]) ? 1 : 0;
     cps[b].active = (a.active == nullptr || a.active[b]) ? 1 : 0;
   }
+  const uint32_t seed_lo = static_cast<uint32_t>(pr.seed & 0xFFFFFFFFull);
+  const uint32_t seed_hi = static_cast<uint32_t>(pr.seed >> 32);
+  float* part = reinterpret_cast<float*>(wsb + ws.part_off);
 
-  // TMA boxes: one CTA's share of a stage, 128 rows x 128 bytes of K (the
-  // 128-byte swizzle span); the kernel's expect-tx byte counts and shared-
-  // memory slots are sized from the same constants.  K beyond d reads as 0.
-  static_assert(kTileBytes == kBlockK * 2 * kBlockM && kTileBytes == kBlockKFp8 * 1 * kHalfN,
-                "TMA box / stage tile mismatch");
-  CUtensorMap tmA, tmA2, tmB;
-  if (fp8) {
-    // h -> h1 + h2 (E4M3) with a power-of-two row scale, in the workspace
-    uint8_t* h1 = wsb + ws.h1_off;
-    uint8_t* h2 = wsb + ws.h2_off;
-    if (!cuda_ok(launch_hidden_split(a.h, h1, h2, reinterpret_cast<float*>(wsb + ws.rinv_off), R, s.d,
-                                     reinterpret_cast<uint32_t*>(wsb + ws.err_off), a.stream),
-                 "hidden-state split launch"))
+  if (head) {
+    // TMA boxes: one CTA's share of a stage, 128 rows x 128 bytes of K (the
+    // 128-byte swizzle span); the kernel's expect-tx byte counts and shared-
+    // memory slots are sized from the same constants.  K beyond d reads as 0.
+    static_assert(kTileBytes == kBlockK * 2 * kBlockM && kTileBytes == kBlockKFp8 * 1 * kHalfN,
+                  "TMA box / stage tile mismatch");
+    CUtensorMap tmA, tmA2, tmB;
+    if (fp8) {
+      // h -> h1 + h2 (E4M3) with a power-of-two row scale, in the workspace
+      uint8_t* h1 = wsb + ws.h1_off;
+      uint8_t* h2 = wsb + ws.h2_off;
+      if (!cuda_ok(launch_hidden_split(a.h, h1, h2, reinterpret_cast<float*>(wsb + ws.rinv_off), R, s.d,
+                                       reinterpret_cast<uint32_t*>(wsb + ws.err_off), a.stream),
+                   "hidden-state split launch"))
+        return DG_ERR_CUDA;
+      const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+      const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
+      if (!encode_2d(&tmA, U8, 1, SW, h1, s.d, R, kBlockKFp8, kBlockM) ||
+          !encode_2d(&tmA2, U8, 1, SW, h2, s.d, R, kBlockKFp8, kBlockM) ||
+          !encode_2d(&tmB, U8, 1, SW, a.E, s.d, s.V, kBlockKFp8, kHalfN))
+        return DG_ERR_CUDA;
+    } else {
+      const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+      const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
+      if (!encode_2d(&tmA, BF, 2, SW, a.h, s.d, R, kBlockK, kBlockM) ||
+          !encode_2d(&tmB, BF, 2, SW, a.E, s.d, s.V, kBlockK, kHalfN))
+        return DG_ERR_CUDA;
+      tmA2 = tmA;  // unused by the bf16 head
+    }
+    if (a.mode == StepMode::kHeadOnly) {
+      // the per-row key records must start empty; without the merge of this
+      // call nothing else clears them
+      if (!cuda_ok(cudaMemsetAsync(row_rec, 0, sizeof(uint32_t) * static_cast<size_t>(R), a.stream),
+                   "record clear"))
+        return DG_ERR_CUDA;
+      part = a.part_out;
+    }
+
+    HeadParams hp;
+    memset(&hp, 0, sizeof(hp));
+    hp.R = R;
+    hp.d = s.d;
+    hp.V = s.V;
+    hp.B = s.B;
+    hp.v_off = a.v_off;
+    hp.split = head_split(R, s.V, s.d, pairs, fp8 ? kBlockKFp8 : kBlockK);
+    hp.seed_lo = seed_lo;
+    hp.seed_hi = seed_hi;
+    // Philox4x32-10 round keys: key + i * (0x9E3779B9, 0xBB67AE85), mod 2^32
+    for (int i = 0; i < 10; ++i) {
+      hp.rk0[i] = seed_lo + static_cast<uint32_t>(i) * 0x9E3779B9u;
+      hp.rk1[i] = seed_hi + static_cast<uint32_t>(i) * 0xBB67AE85u;
+    }
+    hp.e_scale = a.e_scale;
+    hp.row_inv = fp8 ? reinterpret_cast<const float*>(wsb + ws.rinv_off) : nullptr;
+    hp.part = part;
+    hp.err = reinterpret_cast<uint32_t*>(wsb + ws.err_off);
+    hp.logits_out = a.logits;
+    hp.row_rec = row_rec;
+    hp.wait_ns = kDefaultWaitNs;
+    memcpy(hp.cp, cps, sizeof(cps));
+
+    if (t_head_ev_start != nullptr && cudaEventRecord(t_head_ev_start, a.stream) != cudaSuccess)
       return DG_ERR_CUDA;
-    const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
-    const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
-    if (!encode_2d(&tmA, U8, 1, SW, h1, s.d, R, kBlockKFp8, kBlockM) ||
-        !encode_2d(&tmA2, U8, 1, SW, h2, s.d, R, kBlockKFp8, kBlockM) ||
-        !encode_2d(&tmB, U8, 1, SW, a.E, s.d, s.V, kBlockKFp8, kHalfN))
+    if (!cuda_ok(launch_head(fp8, tmA, tmA2, tmB, hp, a.stream), "head kernel launch")) return DG_ERR_CUDA;
+    if (t_head_ev_stop != nullptr && cudaEventRecord(t_head_ev_stop, a.stream) != cudaSuccess)
       return DG_ERR_CUDA;
-  } else {
-    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
-    if (!encode_2d(&tmA, BF, 2, SW, a.h, s.d, R, kBlockK, kBlockM) ||
-        !encode_2d(&tmB, BF, 2, SW, a.E, s.d, s.V, kBlockK, kHalfN))
-      return DG_ERR_CUDA;
-    tmA2 = tmA;  // unused by the bf16 head
   }
-
-  HeadParams hp;
-  memset(&hp, 0, sizeof(hp));
-  hp.R = R;
-  hp.d = s.d;
-  hp.V = s.V;
-  hp.B = s.B;
-  hp.split = head_split(R, s.V, s.d, pairs, fp8 ? kBlockKFp8 : kBlockK);
-  hp.seed_lo = static_cast<uint32_t>(pr.seed & 0xFFFFFFFFull);
-  hp.seed_hi = static_cast<uint32_t>(pr.seed >> 32);
-  // Philox4x32-10 round keys: key + i * (0x9E3779B9, 0xBB67AE85), mod 2^32
-  for (int i = 0; i < 10; ++i) {
-    hp.rk0[i] = hp.seed_lo + static_cast<uint32_t>(i) * 0x9E3779B9u;
-    hp.rk1[i] = hp.seed_hi + static_cast<uint32_t>(i) * 0xBB67AE85u;
-  }
-  hp.e_scale = a.e_scale;
-  hp.row_inv = fp8 ? reinterpret_cast<const float*>(wsb + ws.rinv_off) : nullptr;
-  hp.part = reinterpret_cast<float*>(wsb + ws.part_off);
-  hp.err = reinterpret_cast<uint32_t*>(wsb + ws.err_off);
-  hp.logits_out = a.logits;
-  hp.row_rec = reinterpret_cast<uint32_t*>(wsb + ws.rec_off);
-  hp.wait_ns = kDefaultWaitNs;
-  memcpy(hp.cp, cps, sizeof(cps));
-
-  if (t_head_ev_start != nullptr && cudaEventRecord(t_head_ev_start, a.stream) != cudaSuccess)
-    return DG_ERR_CUDA;
-  if (!cuda_ok(launch_head(fp8, tmA, tmA2, tmB, hp, a.stream), "head kernel launch")) return DG_ERR_CUDA;
-  if (t_head_ev_stop != nullptr && cudaEventRecord(t_head_ev_stop, a.stream) != cudaSuccess)
-    return DG_ERR_CUDA;
+  if (!merge) return DG_OK;
 
   MergeParams mp;
   memset(&mp, 0, sizeof(mp));
   mp.R = R;
   mp.B = s.B;
   mp.V = s.V;
-  mp.P = ws.P;
-  mp.part = hp.part;
+  mp.P = a.mode == StepMode::kMergeOnly ? a.P : ws.P;
+  mp.S = a.mode == StepMode::kMergeOnly ? a.S : 1;
+  mp.part = a.mode == StepMode::kMergeOnly ? a.part_in : part;
   mp.entropy = a.entropy;
   mp.sampled = a.sampled;
   mp.argmax = a.argmax;
@@ -239,9 +271,9 @@ dg_status run_step(const StepArgs& a) {
   mp.accept = a.accept;
   mp.stop = a.stop;
   mp.tickets = reinterpret_cast<uint32_t*>(wsb + ws.tickets_off);
-  mp.row_rec = hp.row_rec;
-  mp.seed_lo = hp.seed_lo;
-  mp.seed_hi = hp.seed_hi;
+  mp.row_rec = row_rec;
+  mp.seed_lo = seed_lo;
+  mp.seed_hi = seed_hi;
   mp.entropy_bound = pr.entropy_bound;
   mp.selection_rule = pr.selection_rule;
   mp.top_k = pr.top_k;
@@ -415,6 +447,42 @@ dg_status dg_denoise_loop(const dg_shape* shape, const dg_params* params, const 
   }
   if (cudaStreamSynchronize(cs) != cudaSuccess) return DG_ERR_CUDA;
   return DG_OK;
+}
+
+int32_t dg_partials_count(const dg_shape* shard_shape) {
+  if (check_shape(shard_shape) != DG_OK) return 0;
+  if (device_sms() <= 0) return 0;
+  const int pairs = head_max_pairs(shard_shape->e_dtype == DG_E_FP8_E4M3);
+  if (pairs <= 0) return 0;
+  return ws_layout(*shard_shape, pairs).P;
+}
+
+dg_status dg_head_partials(const dg_shape* shard_shape, const dg_params* params, int32_t v_offset,
+                           const void* h, const void* E_shard, const float* e_scale_shard,
+                           const int32_t* step_idx, float* partials, void* workspace, size_t ws_bytes,
+                           void* stream) {
+  StepArgs a{shard_shape, params, h, E_shard, e_scale_shard, step_idx, nullptr, nullptr, nullptr, nullptr,
+             nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, workspace, ws_bytes,
+             static_cast<cudaStream_t>(stream)};
+  a.mode = StepMode::kHeadOnly;
+  a.v_off = v_offset;
+  a.part_out = partials;
+  return run_step(a);
+}
+
+dg_status dg_merge_partials(const dg_shape* shape, const dg_params* params, const float* partials,
+                            int32_t shards, int32_t count, const int32_t* step_idx, const uint8_t* has_prev,
+                            const uint8_t* active, int32_t* canvas, int32_t* prev_argmax, uint8_t* accept,
+                            float* entropy, int32_t* sampled, int32_t* argmax, int32_t* stop, void* workspace,
+                            size_t ws_bytes, void* stream) {
+  StepArgs a{shape,   params,  nullptr, nullptr, nullptr, step_idx, has_prev, active, canvas, prev_argmax,
+             accept,  entropy, sampled, argmax,  stop,    nullptr,  workspace, ws_bytes,
+             static_cast<cudaStream_t>(stream)};
+  a.mode = StepMode::kMergeOnly;
+  a.part_in = partials;
+  a.S = shards;
+  a.P = count;
+  return run_step(a);
 }
 
 const char* dg_last_error_message(void) { return t_last_error; }

@@ -76,6 +76,7 @@ struct HeadSplit {
 
 struct HeadParams {
   int32_t R, d, V, B;
+  int32_t v_off;         // vocabulary index of E's first row (vocabulary-sharded step), else 0
   HeadSplit split;
   uint32_t seed_lo, seed_hi;
   const float* e_scale;  // FP8: per-vocabulary-row scale, else null
@@ -91,6 +92,7 @@ struct HeadParams {
 
 struct MergeParams {
   int32_t R, B, V, P;
+  int32_t S;             // shards: records of row r are shard s's [7][R][P] block, s < S
   const float* part;
   float* entropy;
   int32_t* sampled;

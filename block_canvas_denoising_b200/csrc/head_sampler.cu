@@ -250,7 +250,9 @@ DG_DEV void epi_group(const uint32_t* r, int v0, int row, float rinv, float inv_
     dst[0] = make_float4(z[0], z[1], z[2], z[3]);
     dst[1] = make_float4(z[4], z[5], z[6], z[7]);
   }
-  process8(z, v0, inv_tau, c2, ctr1, ctr2, ctr3, p.rk0, p.rk1, thr, have_wm, wm_pre, pt, sc);
+  // z, e_scale and the dump are indexed within this launch's rows of E; the
+  // sampler (Philox counters, token indices) uses the global vocabulary index
+  process8(z, v0 + p.v_off, inv_tau, c2, ctr1, ctr2, ctr3, p.rk0, p.rk1, thr, have_wm, wm_pre, pt, sc);
 }
 
 // Named barrier over the epilogue warps only (barrier 1).
@@ -471,7 +473,7 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         const int hrow = m_t * kPairM + static_cast<int>(rank) * kBlockM + kMmaQuarter * 32 + r;
         const int hb = hrow >> 8;
         uint32_t w[8];
-        philox_words8(static_cast<uint32_t>(n_t * kBlockN + g * 8) >> 2,
+        philox_words8(static_cast<uint32_t>(p.v_off + n_t * kBlockN + g * 8) >> 2,
                       static_cast<uint32_t>(hrow & 255) | (kPurposeGumbel << 16), static_cast<uint32_t>(p.cp[hb].k),
                       static_cast<uint32_t>(hb), p.rk0, p.rk1, w);
         dst[g * 32 + r] = max(max(max(w[0], w[1]), max(w[2], w[3])), max(max(w[4], w[5]), max(w[6], w[7])));

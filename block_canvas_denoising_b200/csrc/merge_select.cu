@@ -76,7 +76,11 @@ merge_select_kernel(const __grid_constant__ MergeParams p) {
   // then a fixed tree over the lanes (lane i absorbs lane i + off)
   Partial a;
   partial_init(a);
-  for (int q = lane; q < p.P; q += 32) partial_merge(a, partial_load(p.part, plane, static_cast<size_t>(row) * p.P + q));
+  const size_t shard_stride = static_cast<size_t>(kPartialFields) * plane;
+  for (int qq = lane; qq < p.S * p.P; qq += 32) {
+    const int s = qq / p.P, q = qq - s * p.P;
+    partial_merge(a, partial_load(p.part + s * shard_stride, plane, static_cast<size_t>(row) * p.P + q));
+  }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
     const Partial o = partial_shfl_down(a, off);

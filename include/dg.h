@@ -237,6 +237,47 @@ dg_status dg_denoise_step_noalloc(const dg_shape* shape, const dg_params* params
                                   uint8_t* accept, float* entropy, int32_t* sampled,
                                   int32_t* argmax, int32_t* stop, void* stream);
 
+/* ---- vocabulary-sharded step ---------------------------------------------
+ * For an embedder split over G GPUs by vocabulary rows (equal shards of
+ * V / G rows, each a multiple of 256): every rank runs dg_head_partials on
+ * its shard, the caller gathers the G record blocks (for example an NCCL
+ * all-gather into a [G][...] buffer), and every rank (or one) runs
+ * dg_merge_partials on all of them.  The result equals dg_denoise_step over
+ * the whole vocabulary: the Philox counters and token indices use the
+ * global vocabulary index; only the float32 merge order of the softmax
+ * partials differs (entropies agree to rounding).  The pages do not describe
+ * a sharded step; this is the data-parallel layout of the same method. */
+
+/* Records per canvas row that dg_head_partials writes for a shard of this
+ * shape on the current device (shape->V = the shard's rows); the records
+ * occupy 7 * B * L * count floats.  0 for an invalid shape. */
+int32_t dg_partials_count(const dg_shape* shard_shape);
+
+/* The fused head and sampler over one shard: E_shard holds vocabulary rows
+ * v_offset .. v_offset + shard_shape->V - 1 (v_offset a multiple of 256),
+ * e_scale_shard their scales (FP8 only).  Writes the per-row partial records
+ * (online softmax, argmax, best Gumbel key) to `partials` (device, 16-byte
+ * aligned, 7 * B * L * dg_partials_count(shard_shape) floats).  step_idx is
+ * a host array as for dg_denoise_step; the workspace is one of
+ * dg_workspace_size(shard_shape) bytes. */
+dg_status dg_head_partials(const dg_shape* shard_shape, const dg_params* params, int32_t v_offset,
+                           const void* h, const void* E_shard, const float* e_scale_shard,
+                           const int32_t* step_idx, float* partials,
+                           void* workspace, size_t ws_bytes, void* stream);
+
+/* Merge `shards` record blocks of `count` records per row each (laid out
+ * [shards][7][B*L][count] as written by dg_head_partials), then selection,
+ * renoise and the stop test as dg_denoise_step does.  shape->V is the whole
+ * vocabulary (the renoise draws from all of it).  The workspace may be the
+ * one the head used (any workspace for the same B). */
+dg_status dg_merge_partials(const dg_shape* shape, const dg_params* params, const float* partials,
+                            int32_t shards, int32_t count, const int32_t* step_idx,
+                            const uint8_t* has_prev, const uint8_t* active,
+                            int32_t* canvas, int32_t* prev_argmax,
+                            uint8_t* accept, float* entropy, int32_t* sampled,
+                            int32_t* argmax, int32_t* stop,
+                            void* workspace, size_t ws_bytes, void* stream);
+
 /* ---- diagnostics (no counterpart on the pages; used by the tests) ---- */
 
 /* Text of the last CUDA runtime error met by a call on this host thread

@@ -108,3 +108,25 @@ def test_embedder_scale_checks(libdg):
 
 def test_workspace_size_zero_for_bad_shape(libdg):
     assert dg.workspace_size(1, 100, 8192) == 0
+
+
+def test_sharded_entry_points_host_checks(libdg):
+    # v_offset must be a multiple of 256; the merge needs at least one shard
+    # and record; all refused before any device work
+    shp = dg._Shape(1, 256, 512, 4096, 0)
+    prm = dg.Params().c()
+    ks = np.zeros(1, np.int32)
+    hp = np.zeros(1, np.uint8)
+    fake = ctypes.c_void_p(256)
+    kp = ks.ctypes.data_as(ctypes.c_void_p)
+    assert libdg.dg_head_partials(ctypes.byref(shp), ctypes.byref(prm), 100, fake, fake, None, kp, fake, fake,
+                                  ctypes.c_size_t(1 << 30), None) == 1
+    assert libdg.dg_head_partials(ctypes.byref(shp), ctypes.byref(prm), -256, fake, fake, None, kp, fake, fake,
+                                  ctypes.c_size_t(1 << 30), None) == 1
+    outs = [fake] * 7
+    assert libdg.dg_merge_partials(ctypes.byref(shp), ctypes.byref(prm), fake, 0, 4, kp,
+                                   hp.ctypes.data_as(ctypes.c_void_p), None, *outs, fake,
+                                   ctypes.c_size_t(1 << 30), None) == 1
+    assert libdg.dg_merge_partials(ctypes.byref(shp), ctypes.byref(prm), fake, 2, 0, kp,
+                                   hp.ctypes.data_as(ctypes.c_void_p), None, *outs, fake,
+                                   ctypes.c_size_t(1 << 30), None) == 1

@@ -68,3 +68,39 @@ def test_reference_arm_on_nonzero_rank_exits_quietly():
                        env=env, capture_output=True, text=True, timeout=300, cwd=ROOT)
     assert r.returncode == 0, r.stderr[-500:]
     assert r.stdout.strip() == ""
+
+
+def _gather_worker(rank, world, port, q):
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                           world_size=world, timeout=timedelta(seconds=60))
+    try:
+        import block_canvas_denoising_b200 as dg
+        local = torch.arange(7 * 4 * 3, dtype=torch.float32).view(7, 4, 3) + 1000.0 * rank
+        out = dg.gather_partials(local)
+        q.put((rank, tuple(out.shape), out[:, 2, 1, 0].tolist(), bool(torch.equal(out[rank], local))))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_vocab_sharded_records_gathered_in_rank_order_on_gloo():
+    # the sharded step's only collective: every rank ends with all ranks'
+    # record blocks, rank r's at index r (the merge's shard order)
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_gather_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = sorted(q.get(timeout=120) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    v = 2 * 12 + 1 * 3 + 0
+    for rank, shape, vals, own in out:
+        assert shape == (2, 7, 4, 3) and own
+        assert vals == [float(v), 1000.0 + v]
