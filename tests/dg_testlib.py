@@ -114,7 +114,7 @@ def compare_with_oracle(g, h_bits, E_bits, step_idx, has_prev, prev_argmax, para
         err = np.abs(zg - z_or).max()
         scale = np.abs(z_or).max()
         info["logit_max_abs_err"] = float(err)
-        info["logit_rel_err"] = float(err / scale)
+        info["logit_rel_err"] = float(err / scale) if scale > 0 else (0.0 if err == 0 else float("inf"))
         assert err <= LOGIT_REL_TOL * scale, (err, scale)
         # argmax margin of the oracle's logits
         top2 = -np.partition(-z_or, 1, axis=1)[:, :2]
