@@ -106,20 +106,10 @@ DG_DEV bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t limit_ns) 
   }
 }
 
-// 2-D tiled TMA load into this CTA's shared memory, completing on `bar`.
-// x is the inner (contiguous) coordinate in elements, y the row.
-DG_DEV void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y,
-                        uint64_t cache_hint) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "l"(cache_hint)
-      : "memory");
-}
-
-// Pair variant (tcgen05 cta_group::2): the copy lands in this CTA's shared
-// memory and completes on `bar`, which may be the peer CTA's barrier (a
-// shared::cluster address from mapa).
+// 2-D tiled TMA load for a tcgen05 cta_group::2 pair: the copy lands in this
+// CTA's shared memory and completes on `bar`, which may be the peer CTA's
+// barrier (a shared::cluster address from mapa).  x is the inner
+// (contiguous) coordinate in elements, y the row.
 DG_DEV void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y,
                              uint64_t cache_hint) {
   asm volatile(
@@ -174,33 +164,13 @@ DG_DEV uint64_t policy_evict_last() {
 }
 
 // ---------------------------------------------------------------------------
-// tcgen05 (5th-generation tensor core, accumulators in tensor memory)
+// tcgen05 (5th-generation tensor core, accumulators in tensor memory), in
+// the pair form (cta_group::2): TMEM is allocated in both CTAs of the pair by
+// one warp of each; the leader issues the MMA over both CTAs' operands.
 // ---------------------------------------------------------------------------
-DG_DEV void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
-               "r"(ncols)
-               : "memory");
-}
-DG_DEV void tmem_relinquish() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-DG_DEV void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-               : "memory");
-}
 DG_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 DG_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// Arrive once on `bar` when every tcgen05 operation issued so far by this
-// thread has completed.
-DG_DEV void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   bar)
-               : "memory");
-}
-
-// Pair forms (cta_group::2): TMEM is allocated in both CTAs of the pair by
-// one warp of each; the leader issues the MMA over both CTAs' operands.
 DG_DEV void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
                "r"(ncols)
@@ -224,21 +194,12 @@ DG_DEV void tc_commit_pair_mc(uint32_t bar, uint16_t cta_mask) {
       : "memory");
 }
 
-// D[tmem of both CTAs] (+)= A[smem of both] * B[smem of both]^T (M = 256 over
-// the pair, N split between the two CTAs' B tiles), bf16, f32 accumulate.
-DG_DEV void tc_mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                             uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// The same pair MMAs with each smem descriptor given as its two 32-bit
-// halves (the low half carries the start address, so stepping along K or to
-// the next stage is one 32-bit add), for an issuing loop with as few
+// D[tmem of both CTAs] (+)= A[smem of both] * B[smem of both]^T (M = 256
+// over the pair, N split between the two CTAs' B tiles), f32 accumulate:
+// kind::f16 with bf16 operands (K = 16 per instruction) or kind::f8f6f4
+// with E4M3 operands (K = 32).  Each smem descriptor is given as its two
+// 32-bit halves (the low half carries the start address, so stepping along
+// K or to the next stage is one 32-bit add), for an issuing loop with as few
 // instructions as possible.
 template <bool kE4M3>
 DG_DEV void tc_mma_pair_lohi(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi, uint32_t b_lo, uint32_t b_hi,
@@ -262,28 +223,6 @@ DG_DEV void tc_mma_pair_lohi(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi, uint
         "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
         : "memory");
   }
-}
-
-// Pair MMA with E4M3 operands (K = 32 per instruction), f32 accumulate.
-DG_DEV void tc_mma_e4m3_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                             uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, f32 accumulate.
-DG_DEV void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                        uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
 }
 
 // Shared-memory matrix descriptor of a K-major tile stored by TMA with the
@@ -316,36 +255,6 @@ __host__ __device__ constexpr uint32_t instr_desc_e4m3_f32(int M, int N) {
   return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-// Issue a load of 32 consecutive f32 columns of this thread's TMEM lane
-// (32x32b shape).  The registers are valid only after tmem_load_wait(r).
-DG_DEV void tmem_load_issue(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr)
-      : "memory");
-}
-
-// Wait for this thread's outstanding TMEM loads; the registers of the last
-// load are tied to the wait so no use is scheduled above it.
-DG_DEV void tmem_load_wait(uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.wait::ld.sync.aligned;"
-      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
-        "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
-        "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),
-        "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
-        "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
-      :
-      : "memory");
-}
-
 // Issue a load of 8 consecutive f32 columns of this thread's TMEM lane.
 DG_DEV void tmem_load8_issue(uint32_t taddr, uint32_t (&r)[8]) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
@@ -360,26 +269,6 @@ DG_DEV void tmem_load8_wait(uint32_t (&r)[8]) {
                  "+r"(r[6]), "+r"(r[7])
                :
                : "memory");
-}
-
-// 32 consecutive f32 columns of this thread's TMEM lane (32x32b shape), with
-// the wait folded into the same statement so no use can move above it.
-DG_DEV void tmem_load_32cols(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr)
-      : "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // ---------------------------------------------------------------------------
@@ -408,41 +297,8 @@ DG_DEV void philox4x32_10(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3, ui
   out[3] = x3;
 }
 
-// The ten round keys of a Philox4x32-10 key (k + i * Weyl constants).
-struct PhiloxKeys {
-  uint32_t k0[10], k1[10];
-};
-DG_DEV PhiloxKeys philox_keys(uint32_t k0, uint32_t k1) {
-  PhiloxKeys k;
-#pragma unroll
-  for (int i = 0; i < 10; ++i) {
-    k.k0[i] = k0;
-    k.k1[i] = k1;
-    k0 += 0x9E3779B9u;
-    k1 += 0xBB67AE85u;
-  }
-  return k;
-}
-DG_DEV void philox4x32_10_rk(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3, const PhiloxKeys& k,
-                             uint32_t (&out)[4]) {
-#pragma unroll
-  for (int i = 0; i < 10; ++i) {
-    const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * x0;
-    const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * x2;
-    const uint32_t y0 = static_cast<uint32_t>(p1 >> 32) ^ x1 ^ k.k0[i];
-    const uint32_t y2 = static_cast<uint32_t>(p0 >> 32) ^ x3 ^ k.k1[i];
-    x1 = static_cast<uint32_t>(p1);
-    x3 = static_cast<uint32_t>(p0);
-    x0 = y0;
-    x2 = y2;
-  }
-  out[0] = x0;
-  out[1] = x1;
-  out[2] = x2;
-  out[3] = x3;
-}
-
-// Same, with the round keys in two arrays (e.g. kernel parameters).
+// Same, with the ten round keys (key + i * Weyl constants) precomputed in
+// two arrays (kernel parameters).
 DG_DEV void philox4x32_10_keys(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3,
                                const uint32_t (&k0)[10], const uint32_t (&k1)[10], uint32_t (&out)[4]) {
 #pragma unroll
