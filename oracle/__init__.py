@@ -14,6 +14,8 @@ Modules:
              entropy-bounded selection, renoise, stop.
   replay  -- the sampler replayed on given float32 logits.
   loop    -- the adaptive loop with final commit.
+  selfcond -- the self-conditioning signal read as the expected embedding
+             (its CUDA side is not built yet).
 
 Parity pins: every function is checked in ``tests/test_oracle_*.py`` against
 something other than itself (closed forms, brute force in exact arithmetic,
@@ -21,10 +23,10 @@ independent library routines, invariants, chi-square).  The composed step has
 no worked example on the pages: its end-to-end values are pinned only through
 its parts.
 """
-from . import flog, loop, philox, replay, step
+from . import flog, loop, philox, replay, selfcond, step
 from .loop import denoise_loop
 from .replay import replay_step
 from .step import Params, denoise_step
 
-__all__ = ["flog", "loop", "philox", "replay", "step", "Params",
+__all__ = ["flog", "loop", "philox", "replay", "selfcond", "step", "Params",
            "denoise_step", "denoise_loop", "replay_step"]
