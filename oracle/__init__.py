@@ -14,6 +14,7 @@ Modules:
              entropy-bounded selection, renoise, stop.
   replay  -- the sampler replayed on given float32 logits.
   loop    -- the adaptive loop with final commit.
+  blocks  -- block-by-block generation (encode & append) over the loop.
   selfcond -- the self-conditioning signal read as the expected embedding
              (its CUDA side is not built yet).
 
@@ -23,10 +24,11 @@ independent library routines, invariants, chi-square).  The composed step has
 no worked example on the pages: its end-to-end values are pinned only through
 its parts.
 """
-from . import flog, loop, philox, replay, selfcond, step
+from . import blocks, flog, loop, philox, replay, selfcond, step
+from .blocks import generate_blocks
 from .loop import denoise_loop
 from .replay import replay_step
 from .step import Params, denoise_step
 
-__all__ = ["flog", "loop", "philox", "replay", "selfcond", "step", "Params",
-           "denoise_step", "denoise_loop", "replay_step"]
+__all__ = ["blocks", "flog", "loop", "philox", "replay", "selfcond", "step", "Params",
+           "denoise_step", "denoise_loop", "generate_blocks", "replay_step"]

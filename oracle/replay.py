@@ -14,7 +14,7 @@ from __future__ import annotations
 import numpy as np
 
 from .flog import gumbel_f32, uniform_f32
-from .step import (Params, argmax_lowest, entropy, gumbel_words, inv_tau_f32,
+from .step import (Params, argmax_lowest, counter_step, entropy, gumbel_words, inv_tau_f32,
                    renoise_tokens, select, stop_flag)
 
 
@@ -47,14 +47,14 @@ def replay_step(z32, *, B: int, L: int, step_idx, has_prev, prev_argmax,
         H = np.empty(L)
         for s0 in range(0, L, slot_chunk):
             s1 = min(L, s0 + slot_chunk)
-            w = gumbel_words(np.arange(s0, s1), b, k, V, params.seed)
+            w = gumbel_words(np.arange(s0, s1), b, counter_step(k, params.block), V, params.seed)
             samp[s0:s1] = np.argmax(key_f32(zc[s0:s1], it, w), axis=1)
             H[s0:s1] = entropy(zc[s0:s1].astype(np.float64) * np.float64(it))
         if entropy_in is not None:
             H = np.asarray(entropy_in[i * L:(i + 1) * L], dtype=np.float64)
         amax = argmax_lowest(zc)
         acc, _, om = select(H, params.entropy_bound, params.selection_rule, params.top_k)
-        noise = renoise_tokens(b, k, L, V, params.seed)
+        noise = renoise_tokens(b, counter_step(k, params.block), L, V, params.seed)
         canvas = np.where(acc == 1, samp, noise).astype(np.int32)
         st, _ = stop_flag(H, amax, prev_argmax[b * L:(b + 1) * L], bool(has_prev[b]),
                           params.stop_entropy)

@@ -38,6 +38,7 @@ STOP_ENTROPY = 0.005  # adaptive-stop mean-entropy threshold
 
 PURPOSE_GUMBEL = 0
 PURPOSE_RENOISE = 1
+PURPOSE_INIT = 3      # the noise canvas a block starts from
 
 
 # selection rules (the default is this project's reading of the pages)
@@ -56,6 +57,17 @@ class Params:
     seed: int = 1234
     selection_rule: int = SELECT_CUMSUM
     top_k: int = 1
+    block: int = 0    # index of the canvas block in a block-by-block generation
+
+
+def counter_step(k: int, block: int = 0) -> int:
+    """Third Philox counter word of step k of canvas block ``block``:
+    k | block << 16, so every block draws its own streams (k < 2^16).
+    [Report] Figure 4: generation proceeds block after block, each block
+    denoised from fresh noise; a single block is block 0 (word = k)."""
+    if not (0 <= k < 1 << 16 and 0 <= block < 1 << 16):
+        raise ValueError("step or block index out of range")
+    return int(k) | (int(block) << 16)
 
 
 # --------------------------------------------------------------------------
@@ -285,6 +297,21 @@ def renoise_tokens(b: int, k: int, L: int, V: int, seed: int) -> np.ndarray:
     return ((r * np.uint64(V)) >> np.uint64(32)).astype(np.int32)
 
 
+def initial_canvas(b: int, block: int, L: int, V: int, seed: int) -> np.ndarray:
+    """The all-noise canvas block ``block`` of canvas b starts from, int32 [L].
+
+    [Report] Figure 4: a block is denoised from pure noise; Figure 3: the
+    noise is uniform over the vocabulary.  Philox counter
+    (0, slot | 3 << 16, block << 16, b), lane 0, token = (r * V) >> 32.
+    """
+    k0, k1 = split_seed(seed)
+    slots = np.arange(L, dtype=np.uint64)
+    o = philox4x32_10(np.uint64(0), slots | np.uint64(PURPOSE_INIT << 16),
+                      np.uint64(counter_step(0, block)), np.uint64(b), k0, k1)
+    r = o[0].astype(np.uint64)
+    return ((r * np.uint64(V)) >> np.uint64(32)).astype(np.int32)
+
+
 def stop_flag(H, argmax, prev_argmax, has_prev: bool, stop_entropy: float = STOP_ENTROPY):
     """Adaptive stop of one canvas.
 
@@ -310,12 +337,15 @@ def denoise_step(h_bits, *, E_bits=None, q=None, s=None, B: int, L: int = 256,
     ``h_bits`` is [B*L, d] bf16 bits (row b*L + s is slot s of canvas b).
     ``step_idx`` [B], ``has_prev`` [B], ``prev_argmax`` [B*L].
     Returns a dict of per-slot arrays over the chosen canvases (rows in
-    canvas order) and per-canvas arrays, plus the decision margins.
+    canvas order) and per-canvas arrays, plus the decision margins
+    (``gumbel_margin``: best minus second Gumbel key; ``argmax_margin``:
+    best minus second logit; ``order_margin`` and ``stop_margin`` per
+    canvas, see ``select`` and ``stop_flag``).
     """
     V = (E_bits if E_bits is not None else q).shape[0]
     canvases = list(range(B)) if canvases is None else [int(c) for c in canvases]
-    out = {k: [] for k in ("entropy", "sampled", "argmax", "accept", "canvas",
-                           "gumbel_margin", "stop", "order_margin", "stop_margin", "n_accept")}
+    out = {k: [] for k in ("entropy", "sampled", "argmax", "accept", "canvas", "gumbel_margin",
+                           "argmax_margin", "stop", "order_margin", "stop_margin", "n_accept")}
     for b in canvases:
         k = int(step_idx[b])
         tau = temperature(k, params.tau0, params.tau1, params.max_steps)
@@ -324,26 +354,29 @@ def denoise_step(h_bits, *, E_bits=None, q=None, s=None, B: int, L: int = 256,
         samp = np.empty(L, dtype=np.int32)
         gm = np.empty(L)
         amax = argmax_lowest(z)
+        top2 = -np.partition(-z, 1, axis=1)[:, :2]
+        amargin = top2[:, 0] - top2[:, 1]
         for s0 in range(0, L, slot_chunk):
             s1 = min(L, s0 + slot_chunk)
             x = z[s0:s1] / tau
             H[s0:s1] = entropy(x)
-            w = gumbel_words(np.arange(s0, s1), b, k, V, params.seed)
+            w = gumbel_words(np.arange(s0, s1), b, counter_step(k, params.block), V, params.seed)
             samp[s0:s1], gm[s0:s1] = gumbel_sample(x, w)
         acc, n, om = select(H, params.entropy_bound, params.selection_rule, params.top_k)
-        noise = renoise_tokens(b, k, L, V, params.seed)
+        noise = renoise_tokens(b, counter_step(k, params.block), L, V, params.seed)
         canvas = np.where(acc == 1, samp, noise).astype(np.int32)
         st, sm = stop_flag(H, amax, prev_argmax[b * L:(b + 1) * L], bool(has_prev[b]),
                            params.stop_entropy)
         for key, val in (("entropy", H), ("sampled", samp), ("argmax", amax),
-                         ("accept", acc), ("canvas", canvas), ("gumbel_margin", gm)):
+                         ("accept", acc), ("canvas", canvas), ("gumbel_margin", gm),
+                         ("argmax_margin", amargin)):
             out[key].append(val)
         out["stop"].append(st)
         out["order_margin"].append(om)
         out["stop_margin"].append(sm)
         out["n_accept"].append(n)
     res = {key: np.concatenate(out[key]) for key in
-           ("entropy", "sampled", "argmax", "accept", "canvas", "gumbel_margin")}
+           ("entropy", "sampled", "argmax", "accept", "canvas", "gumbel_margin", "argmax_margin")}
     res["stop"] = np.array(out["stop"], dtype=np.int32)
     res["order_margin"] = np.array(out["order_margin"])
     res["stop_margin"] = np.array(out["stop_margin"])

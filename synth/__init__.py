@@ -26,7 +26,7 @@ import numpy as np
 __all__ = [
     "bf16_bits_from_f32", "bf16_bits_to_f32", "normal_bf16", "hidden_normal",
     "embedder_normal", "canvas_uniform", "step_indices_uniform",
-    "quantize_e4m3_rows", "e4m3_bits_from_f32", "loop_targets", "loop_hidden",
+    "quantize_e4m3_rows", "e4m3_bits_from_f32", "loop_targets", "loop_hidden", "block_targets",
 ]
 
 # Rows generated per independent random stream.  Each chunk of rows draws from
@@ -201,3 +201,20 @@ def loop_hidden(k: int, y: np.ndarray, E_bits_bf16: np.ndarray, seed: int = 4) -
     noise = g.standard_normal((len(y), d))
     h = (k / 12.0) * 3.0 * Ey / norm * math.sqrt(d) + noise
     return bf16_bits_from_f32(h.astype(np.float32))
+
+
+def block_targets(j: int, committed: np.ndarray, L: int, V: int, B: int = 1, seed: int = 3) -> np.ndarray:
+    """Targets y[B*L] of the stand-in hidden states of canvas block j in a
+    block-by-block generation.
+
+    Block 0 takes ``loop_targets``; block j >= 1 derives its targets from
+    the block committed just before it, y_i = (c_i * 7919 + 104729 (i + 1)
+    + j) mod V, so every block depends on what the previous one committed.
+    (A stand-in for the model conditioning the next block on the appended
+    context; the pages give no model to run.)
+    """
+    if j == 0:
+        return loop_targets(L, V, seed=seed, B=B)
+    c = np.asarray(committed[j - 1], dtype=np.int64)
+    i = np.arange(B * L, dtype=np.int64)
+    return ((c * 7919 + 104729 * (i + 1) + j) % V).astype(np.int32)

@@ -81,7 +81,8 @@ def run_step(h_bits, E_bits, step_idx, has_prev, prev_argmax, canvas0, params, *
 
 def oparams(p) -> OParams:
     return OParams(tau0=p.tau0, tau1=p.tau1, max_steps=p.max_steps, entropy_bound=p.entropy_bound,
-                   stop_entropy=p.stop_entropy, seed=p.seed, selection_rule=p.selection_rule, top_k=p.top_k)
+                   stop_entropy=p.stop_entropy, seed=p.seed, selection_rule=p.selection_rule, top_k=p.top_k,
+                   block=p.block)
 
 
 def rows_of(canvases, L=256):
@@ -120,7 +121,7 @@ def compare_with_oracle(g, h_bits, E_bits, step_idx, has_prev, prev_argmax, para
         top2 = -np.partition(-z_or, 1, axis=1)[:, :2]
         amargin = top2[:, 0] - top2[:, 1]
     else:
-        amargin = np.full(n, np.inf)
+        amargin = ora["argmax_margin"]
 
     # entropy
     herr = np.abs(g["entropy"][rows].astype(np.float64) - ora["entropy"]).max()
