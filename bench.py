@@ -10,11 +10,17 @@ The embedder (1.48 GB) is far larger than the 126 MB L2, so every step
 streams it from HBM; no flush is needed.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                  [--e-dtype fp8]
+                  [--e-dtype fp8] [--batch B]
 
 ``--e-dtype fp8`` times the FP8-E4M3 embedder variant instead (E quantised
 per row to E4M3 codes with a float32 scale, h still bf16); the default line
-is the bf16 workload.
+is the bf16 workload.  ``--batch B`` runs B independent canvases per step
+(the batched configuration: 2048 rows at B = 8, 8192 at B = 32), each with
+its own step index drawn uniformly from [0, 47] (seed 5) and advanced by one
+every step; at B >= 8 the step is bound by the tensor cores and the roofline
+object says so.  The default B = 1 line also reports the adaptive loop run
+once, untimed, at the production shape on the synthetic stand-in hidden
+states (the step at which it stops).
 
 For N > 1 launch with torch.distributed.run; each rank runs its own canvas
 (replicas, no data-path collective): weak scaling.  ``--impl reference``
@@ -40,7 +46,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = ("denoise-step µs & canvas slots/s at B=1, 256×2816×262144 bf16; "
           "% of roofline")
-B, L, D, V = 1, 256, 2816, 262144
+L, D, V = 256, 2816, 262144
 KS = (0, 23, 47)
 REF_BUDGET_S = 90.0      # wall-clock cap of the oracle's timed steps
 SOAK_S = 1.0             # untimed steady-load run before the timed region
@@ -58,6 +64,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e-dtype", default="bf16", choices=("bf16", "fp8"))
+    ap.add_argument("--batch", type=int, default=1, help="canvases per GPU per step")
+    ap.add_argument("--no-loop", action="store_true", help="skip the untimed production-shape loop run")
     return ap.parse_args()
 
 
@@ -180,25 +188,6 @@ def oracle_canvas_step(h_bits, E_bits, k):
     return time.perf_counter() - t0
 
 
-def oracle_rows_step(h_bits, E_bits, k, rows: int):
-    """The oracle's per-slot path (logits, entropy, argmax, Gumbel draw) on
-    ``rows`` slots plus its per-canvas selection / renoise / stop on them."""
-    from oracle import step as S
-    t0 = time.perf_counter()
-    tau = S.temperature(k)
-    z = S.logits(h_bits[:rows], E_bits=E_bits)
-    x = z / tau
-    H = S.entropy(x)
-    amax = S.argmax_lowest(z)
-    w = S.gumbel_words(np.arange(rows), 0, k, V, seed=1234)
-    samp, _ = S.gumbel_sample(x, w)
-    acc, _, _ = S.select(H)
-    noise = S.renoise_tokens(0, k, rows, V, 1234)
-    np.where(acc == 1, samp, noise)
-    S.stop_flag(H, amax, amax, False)
-    return time.perf_counter() - t0
-
-
 def threads_used() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -236,38 +225,79 @@ def init_dist():
 
 
 def run_reference(args):
+    """The CPU oracle on the same workload: full B = 1 steps (all 256 slots
+    over the whole vocabulary, then selection, renoise and stop), timed one
+    by one; at most REF_BUDGET_S seconds of timed steps are run and the line
+    states how many."""
     world, rank, _ = init_dist()
     if world > 1 and rank != 0:
         return 0
     import synth
     E = synth.embedder_normal(V, D, seed=1)
-    h = synth.hidden_normal(B, L, D, seed=2)
-    rows = 32
+    h = synth.hidden_normal(1, L, D, seed=2)
     for i in range(max(0, min(args.warmup, 1))):
-        oracle_rows_step(h, E, KS[i % 3], rows)
-    # each oracle step costs seconds: time at most REF_BUDGET_S of them
+        oracle_canvas_step(h, E, KS[i % 3])
     times = []
     t_start = time.perf_counter()
     for i in range(args.steps):
-        times.append(oracle_rows_step(h, E, KS[i % 3], rows))
+        times.append(oracle_canvas_step(h, E, KS[i % 3]))
         if time.perf_counter() - t_start > REF_BUDGET_S:
             break
     t = sum(times) / len(times)
-    val = rows / t
+    val = L / t
     line = {
         "impl": "reference", "metric": METRIC, "value": val, "unit": "slots/s",
         "n_gpus": args.gpus, "steps": len(times), "steps_requested": args.steps,
-        "warmup": args.warmup, "ms_per_step": t * 1e3 * (L / rows), "higher_is_better": True, "scaling": "weak",
+        "warmup": min(args.warmup, 1), "warmup_requested": args.warmup,
+        "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": "B=1 canvas, L=256, d=2816, V=262144, bf16 inputs, k cycling 0/23/47",
                    "global_batch": 1, "seq_len": L, "parallelism": "cpu oracle"},
         "cpu_baseline": {"value": val, "unit": "slots/s", "cores": threads_used(), "kind": "oracle",
-                         "sample": f"{rows} of 256 slots per step (full vocabulary), "
-                                   "plus selection/renoise/stop on them"},
+                         "sample": f"{len(times)} full B=1 steps (256 slots, whole vocabulary, selection, "
+                                   f"renoise and stop); timed steps capped at {REF_BUDGET_S:.0f} s"},
         "e2e": {"value": val, "unit": "slots/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def loop_report(dg, E, E_bits, e_scale, fp8, ws_dtype, torch):
+    """The adaptive loop once at the production shape (B = 1), untimed: the
+    synthetic stand-in hidden states of the loop configuration (signal
+    growing with k, targets seed 3, noise seed 4 + k), generated on the host
+    each step and copied in.  Returns the step count at stop with the
+    per-step mean entropy and accepted slots."""
+    import synth
+    y = synth.loop_targets(L, V, seed=3)
+    h_buf = torch.empty((L, D), dtype=torch.bfloat16, device="cuda")
+    canvas = torch.from_numpy(synth.canvas_uniform(1, L, V, seed=0)).cuda()
+    prev = torch.zeros(L, dtype=torch.int32, device="cuda")
+    hp = np.zeros(1, np.uint8)
+    acc = torch.zeros(L, dtype=torch.uint8, device="cuda")
+    ent = torch.zeros(L, dtype=torch.float32, device="cuda")
+    samp = torch.zeros(L, dtype=torch.int32, device="cuda")
+    amax = torch.zeros(L, dtype=torch.int32, device="cuda")
+    stop = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = dg.Workspace(1, D, V, ws_dtype)
+    trace = []
+
+    def hidden(k, canvas_t, h_t):
+        if trace:   # the previous step's results are final once this runs
+            trace[-1]["mean_entropy"] = float(ent.mean())
+            trace[-1]["accepted"] = int(acc.sum())
+        h_t.copy_(torch.from_numpy(synth.loop_hidden(k, y, E_bits, seed=4).view(np.int16)).view(torch.bfloat16))
+        trace.append({"k": int(k)})
+
+    steps = dg.denoise_loop(E, hidden, h_buf, canvas, prev, hp, acc, ent, samp, amax, stop, ws,
+                            dg.Params(), e_scale=e_scale)
+    torch.cuda.synchronize()
+    trace[-1]["mean_entropy"] = float(ent.mean())
+    trace[-1]["accepted"] = int(acc.sum())
+    match = float((canvas.cpu().numpy() == y).mean())
+    return {"steps_at_stop": int(steps[0]), "stopped_early": bool(int(steps[0]) < 48),
+            "per_step": trace, "committed_equals_targets": match,
+            "workload": "B=1, L=256, d=2816, V=262144, stand-in h_i = (k/12) 3 E[y_i]/|E[y_i]| sqrt(d) + N(0,1)"}
 
 
 def main():
@@ -294,7 +324,10 @@ def main():
         dist.barrier()
     dg.lib()
 
-    # ---- inputs: one canvas per rank; the embedder is shared model weights
+    B = int(args.batch)
+    if not 1 <= B <= 256:
+        raise SystemExit("--batch must be in [1, 256]")
+    # ---- inputs: B canvases per rank; the embedder is shared model weights
     h_seed, philox_seed = rank_seeds(rank)
     E_bits = synth.embedder_normal(V, D, seed=1)
     h_bits = synth.hidden_normal(B, L, D, seed=h_seed)
@@ -316,14 +349,20 @@ def main():
                samp=torch.zeros(R, dtype=torch.int32, device="cuda"),
                amax=torch.zeros(R, dtype=torch.int32, device="cuda"),
                stop=torch.zeros(B, dtype=torch.int32, device="cuda"))
-    ws = dg.Workspace(B, D, V, dg.E_FP8_E4M3 if fp8 else dg.E_BF16)
+    ws_dtype = dg.E_FP8_E4M3 if fp8 else dg.E_BF16
+    ws = dg.Workspace(B, D, V, ws_dtype)
     params = dg.Params(seed=philox_seed)
     stream = torch.cuda.current_stream()
+    # step indices: B = 1 cycles 0 / 23 / 47; a batch draws one per canvas
+    # (uniform in [0, 47], seed 5) and advances each by one per step
+    k0 = synth.step_indices_uniform(B, 48, seed=5) if B > 1 else None
+    ks_of = [[KS[i % 3]] if B == 1 else [int((k0[b] + i) % 48) for b in range(B)] for i in range(3 * 48)]
+    hp_first, hp_rest = [0] * B, [1] * B
 
     def step(i, h_in):
-        dg.denoise_step(h_in, E, [KS[i % 3]], [1 if i > 0 else 0], dev["canvas"], dev["prev"],
-                        dev["acc"], dev["ent"], dev["samp"], dev["amax"], dev["stop"], ws, params,
-                        e_scale=e_scale)
+        dg.denoise_step(h_in, E, ks_of[i % len(ks_of)], hp_rest if i > 0 else hp_first, dev["canvas"],
+                        dev["prev"], dev["acc"], dev["ent"], dev["samp"], dev["amax"], dev["stop"], ws,
+                        params, e_scale=e_scale)
 
     def timed_region(K):
         ev_h = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -415,42 +454,62 @@ def main():
     e2e_ms = e2e_total / K2
     e2e_value = world * B * L / (e2e_ms / 1e3)
 
+    loop = None
+    if B == 1 and world == 1 and not args.no_loop:
+        loop = loop_report(dg, E, E_bits, e_scale, fp8, ws_dtype, torch)
+
     if rank == 0:
         pk, pk_kind = peaks()
         e_bytes = 1 if fp8 else 2
         alg_bytes = V * D * e_bytes + R * D * 2
-        achieved = alg_bytes / (head_ms / 1e3) / 1e9
-        traffic, _ = recorded_traffic() if not fp8 else (None, None)
+        traffic, _ = recorded_traffic() if (not fp8 and B == 1) else (None, None)
         # FP8: two E4M3 MMAs per K step at twice the bf16 rate (nominal
         # ratio): the same tensor time as 2 R D V bf16 flops
         flops = 2.0 * R * D * V
+        t_hbm = alg_bytes / (pk["hbm_gbs"] * 1e9)
+        t_tc = flops / (pk["bf16_tflops"] * 1e12)
+        gbs = alg_bytes / (head_ms / 1e3) / 1e9
+        tflops = flops / (head_ms / 1e3) / 1e12
+        if t_tc > 1.2 * t_hbm:     # the batched step: a dense contraction bound by the tensor cores
+            roof = {"bound": "tensor", "achieved": tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": tflops / pk["bf16_tflops"], "traffic": traffic,
+                    "peak_kind": f"{pk_kind} (burst bf16 GEMM)",
+                    "frac_of_sustained": tflops / pk["bf16_tflops_sustained"],
+                    "sustained_peak": pk["bf16_tflops_sustained"],
+                    "hbm_gbs": gbs}
+        else:
+            roof = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "frac": gbs / pk["hbm_gbs"], "traffic": traffic, "peak_kind": pk_kind,
+                    "tensor_tflops": tflops, "tensor_frac": tflops / pk["bf16_tflops"]}
+        roof.update({"kernel": "head_sampler_kernel", "kernel_us": head_ms * 1e3,
+                     "algorithmic_bytes": alg_bytes, "flops": flops,
+                     "step_roofline_us": max(t_hbm, t_tc) * 1e6,
+                     "step_frac": max(t_hbm, t_tc) * 1e3 / ms_per_step})
+        if B == 1:
+            k_desc = "k cycling 0/23/47"
+        else:
+            k_desc = "per-canvas k uniform in [0,47] (seed 5), +1 per step"
+        wl = (f"B={B} canvas{'es' if B > 1 else ''} ({R} rows) per GPU, d=2816, V=262144, "
+              + ("bf16 h, E4M3 embedder with per-row float32 scale, " if fp8 else "bf16 h and E, ") + k_desc)
         line = {
             "metric": METRIC, "value": value, "unit": "slots/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "e4m3 (h split in two E4M3 terms)" if fp8 else "bf16",
             "data": "synthetic",
-            "config": {"workload": ("B=1 canvas (256 slots) per GPU, d=2816, V=262144, bf16 h, "
-                                    "E4M3 embedder with per-row float32 scale, k cycling 0/23/47") if fp8 else
-                                   ("B=1 canvas (256 slots) per GPU, d=2816, V=262144, bf16 h and E, "
-                                    "k cycling 0/23/47"),
-                       "global_batch": world * B, "seq_len": L, "parallelism": f"replicas x{world}",
+            "config": {"workload": wl, "global_batch": world * B, "seq_len": L,
+                       "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2 (E = %.2f GB streamed each step)" % (V * D * e_bytes / 1e9)},
             "us_per_step": ms_per_step * 1e3,
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
-                         "peak_kind": pk_kind, "kernel": "head_sampler_kernel",
-                         "kernel_us": head_ms * 1e3,
-                         "tensor_tflops": flops / (head_ms / 1e3) / 1e12,
-                         "tensor_frac": flops / (head_ms / 1e3) / 1e12 / pk["bf16_tflops"],
-                         "step_roofline_us": max(alg_bytes / (pk["hbm_gbs"] * 1e9),
-                                                 flops / (pk["bf16_tflops"] * 1e12)) * 1e6},
+            "roofline": roof,
             "clocks": clocks,
             "e2e": {"value": e2e_value, "unit": "slots/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": (3 if fp8 else 2) * args.steps,
         }
-        if world == 1 and not args.no_cpu_baseline and not fp8:
+        if loop is not None:
+            line["loop"] = loop
+        if world == 1 and B == 1 and not args.no_cpu_baseline and not fp8:
             t_cpu = oracle_canvas_step(h_bits, E_bits, 0)
             line["cpu_baseline"] = {"value": L / t_cpu, "unit": "slots/s", "cores": threads_used(),
                                     "kind": "oracle",

@@ -16,9 +16,10 @@ import numpy as np
 
 __all__ = ["DGError", "Params", "lib", "workspace_size", "Workspace", "denoise_step",
            "debug_logits", "device_status", "denoise_loop", "debug_gumbel",
-           "selftest_bounded_wait", "set_head_events", "denoise_step_noalloc", "STATUS", "E_BF16", "E_FP8_E4M3",
+           "selftest_bounded_wait", "set_head_events", "denoise_step_noalloc", "noalloc_status",
+           "noalloc_selftest_bounded_wait", "STATUS", "E_BF16", "E_FP8_E4M3",
            "SELECT_CUMSUM", "SELECT_MI", "SELECT_TOPK", "partials_count", "head_partials", "merge_partials",
-           "gather_partials"]
+           "gather_partials", "init_canvas", "generate_blocks"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdg.so")
@@ -45,7 +46,8 @@ class _Shape(ctypes.Structure):
 class _Params(ctypes.Structure):
     _fields_ = [("tau0", ctypes.c_double), ("tau1", ctypes.c_double), ("max_steps", ctypes.c_int32),
                 ("entropy_bound", ctypes.c_double), ("stop_entropy", ctypes.c_double),
-                ("seed", ctypes.c_uint64), ("selection_rule", ctypes.c_int32), ("top_k", ctypes.c_int32)]
+                ("seed", ctypes.c_uint64), ("selection_rule", ctypes.c_int32), ("top_k", ctypes.c_int32),
+                ("block", ctypes.c_int32)]
 
 
 SELECT_CUMSUM = 0
@@ -55,6 +57,8 @@ SELECT_TOPK = 2
 
 _HIDDEN_FN = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
                               ctypes.c_void_p, ctypes.c_void_p)
+_BLOCK_HIDDEN_FN = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p,
+                                    ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p)
 
 
 @dataclass
@@ -68,11 +72,12 @@ class Params:
     seed: int = 1234
     selection_rule: int = SELECT_CUMSUM
     top_k: int = 1
+    block: int = 0
 
     def c(self) -> _Params:
         return _Params(self.tau0, self.tau1, self.max_steps, self.entropy_bound,
                        self.stop_entropy, int(self.seed) & 0xFFFFFFFFFFFFFFFF,
-                       int(self.selection_rule), int(self.top_k))
+                       int(self.selection_rule), int(self.top_k), int(self.block))
 
 
 _lib = None
@@ -105,7 +110,16 @@ def lib() -> ctypes.CDLL:
         L.dg_set_head_events.argtypes = [P, P]
         L.dg_denoise_step_noalloc.argtypes = step_args + [P]
         L.dg_denoise_step_noalloc.restype = ctypes.c_int
+        L.dg_noalloc_status.argtypes = [P]
+        L.dg_noalloc_status.restype = ctypes.c_int
+        L.dg_noalloc_selftest_bounded_wait.argtypes = [ctypes.c_uint64, P]
+        L.dg_noalloc_selftest_bounded_wait.restype = ctypes.c_int
         L.dg_last_error_message.restype = ctypes.c_char_p
+        L.dg_init_canvas.argtypes = [ctypes.POINTER(_Shape), ctypes.POINTER(_Params), P, P]
+        L.dg_init_canvas.restype = ctypes.c_int
+        L.dg_generate_blocks.argtypes = [ctypes.POINTER(_Shape), ctypes.POINTER(_Params), P, P, ctypes.c_int32,
+                                         _BLOCK_HIDDEN_FN, P, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+        L.dg_generate_blocks.restype = ctypes.c_int
         L.dg_partials_count.restype = ctypes.c_int32
         L.dg_partials_count.argtypes = [ctypes.POINTER(_Shape)]
         L.dg_head_partials.restype = ctypes.c_int
@@ -207,7 +221,8 @@ def denoise_step_noalloc(h, E, step_idx, has_prev, canvas, prev_argmax, accept, 
                          stream=None) -> None:
     """``dg_denoise_step_noalloc``: the same step without a caller workspace,
     for callers that cannot allocate device memory (the scratch is a fixed
-    8 MiB array inside the library; calls must not overlap on the GPU)."""
+    8 MiB array inside the library; calls must not overlap on the GPU; a
+    device-side fault is reported by ``noalloc_status``)."""
     B = int(len(step_idx))
     R, d = h.shape
     V = E.shape[0]
@@ -223,6 +238,18 @@ def denoise_step_noalloc(h, E, step_idx, has_prev, canvas, prev_argmax, accept, 
         None if act is None else act.ctypes.data_as(ctypes.c_void_p),
         _ptr(canvas), _ptr(prev_argmax), _ptr(accept), _ptr(entropy), _ptr(sampled),
         _ptr(argmax), _ptr(stop), _stream(stream)), "dg_denoise_step_noalloc")
+
+
+def noalloc_status(stream=None) -> int:
+    """Synchronise and read/clear the fault latch of the allocation-free
+    step's scratch array on the current device (0 = no fault)."""
+    return int(lib().dg_noalloc_status(_stream(stream)))
+
+
+def noalloc_selftest_bounded_wait(limit_ns: int, stream=None) -> int:
+    """The bounded-wait self test against the allocation-free step's latch;
+    returns the status it leaves (6 = timed out as designed)."""
+    return int(lib().dg_noalloc_selftest_bounded_wait(ctypes.c_uint64(limit_ns), _stream(stream)))
 
 
 def debug_logits(h, E, step_idx, has_prev, canvas, prev_argmax, accept, entropy, sampled, argmax,
@@ -274,6 +301,55 @@ def denoise_loop(E, hidden_fn, h_buf, canvas, prev_argmax, has_prev, accept, ent
         ctypes.c_size_t(ws.nbytes), _stream(stream))
     if code != 0:
         err = DGError(code, "dg_denoise_loop")
+        if errors:
+            raise err from errors[0]
+        raise err
+    return steps
+
+
+def init_canvas(canvas, B: int, V: int, params: Params = Params(), d: int = 64, stream=None) -> None:
+    """Fill ``canvas`` (int32 CUDA tensor [B*256]) with the uniform noise
+    block ``params.block`` starts from (``dg_init_canvas``)."""
+    shp = _shape(B, d, V, E_BF16, L=int(canvas.numel()) // max(B, 1))
+    prm = params.c()
+    _check(lib().dg_init_canvas(ctypes.byref(shp), ctypes.byref(prm), _ptr(canvas), _stream(stream)),
+           "dg_init_canvas")
+
+
+def generate_blocks(E, hidden_fn, n_blocks: int, h_buf, blocks, canvas, prev_argmax, accept, entropy, sampled,
+                    argmax, stop, ws: Workspace, params: Params = Params(), e_scale=None, stream=None):
+    """Block-by-block generation (``dg_generate_blocks``).
+
+    ``hidden_fn(j, k, canvas_tensor, committed, h_buf)`` fills ``h_buf``
+    for step k of block j on the current stream; ``committed`` is the view
+    ``blocks[:j]`` of the blocks committed so far.  ``blocks`` is an int32
+    CUDA tensor [n_blocks, B*256].  Returns the host int32 array of steps
+    taken, [n_blocks, B]."""
+    R, d = h_buf.shape
+    B = int(len(stop))
+    V = E.shape[0]
+    e_dtype = E_BF16 if e_scale is None else E_FP8_E4M3
+    shp = _shape(B, d, V, e_dtype, L=R // B)
+    prm = params.c()
+    steps = np.zeros((n_blocks, B), np.int32)
+    errors = []
+
+    def cb(j, k, canvas_ptr, committed_ptr, h_ptr, user, stream_ptr):
+        try:
+            hidden_fn(int(j), int(k), canvas, blocks[:int(j)], h_buf)
+            return 0
+        except Exception as exc:  # reported as DG_ERR_CALLBACK
+            errors.append(exc)
+            return 1
+
+    cfn = _BLOCK_HIDDEN_FN(cb)
+    code = lib().dg_generate_blocks(
+        ctypes.byref(shp), ctypes.byref(prm), _ptr(E), _ptr(e_scale), ctypes.c_int32(n_blocks), cfn, None,
+        _ptr(h_buf), _ptr(blocks), steps.ctypes.data_as(ctypes.c_void_p), _ptr(canvas), _ptr(prev_argmax),
+        _ptr(accept), _ptr(entropy), _ptr(sampled), _ptr(argmax), _ptr(stop), _ptr(ws.buf),
+        ctypes.c_size_t(ws.nbytes), _stream(stream))
+    if code != 0:
+        err = DGError(code, "dg_generate_blocks")
         if errors:
             raise err from errors[0]
         raise err

@@ -16,8 +16,9 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libdg.so")
 
-SOURCES = ["dg_api.cu", "head_sampler.cu", "hidden_split.cu", "merge_select.cu", "diagnostics.cu", "noalloc.cu"]
-HEADERS = ["dg_device.cuh", "dg_internal.h"]
+SOURCES = ["dg_api.cu", "head_sampler.cu", "hidden_split.cu", "merge_select.cu", "diagnostics.cu", "noalloc.cu",
+           "blocks.cu"]
+HEADERS = ["dg_device.cuh", "dg_internal.h", "per_device.h"]
 
 
 def nvcc_path() -> str:

@@ -73,6 +73,8 @@ dg_status check_params(const dg_params* p) {
   if (!(p->stop_entropy >= 0.0 && p->stop_entropy < 1e300)) return DG_ERR_INVALID_ARG;
   if (p->selection_rule < DG_SELECT_CUMSUM || p->selection_rule > DG_SELECT_TOPK) return DG_ERR_INVALID_ARG;
   if (p->selection_rule == DG_SELECT_TOPK && (p->top_k < 1 || p->top_k > 256)) return DG_ERR_INVALID_ARG;
+  // the Philox counter's step word is k | block << 16
+  if (p->max_steps > 65536 || p->block < 0 || p->block > 65535) return DG_ERR_INVALID_ARG;
   return DG_OK;
 }
 
@@ -136,7 +138,9 @@ struct StepArgs {
   int32_t S = 1, P = 0;           // merge only
 };
 
-dg_status run_step(const StepArgs& a) {
+// Every check of a step's arguments except those of the workspace: shape,
+// parameters, pointers and their alignment, step indices, the device.
+dg_status check_step_inputs(const StepArgs& a) {
   dg_status st = check_shape(a.shape);
   if (st != DG_OK) return st;
   if ((st = check_params(a.params)) != DG_OK) return st;
@@ -144,7 +148,7 @@ dg_status run_step(const StepArgs& a) {
   const dg_params& pr = *a.params;
   const bool head = a.mode != StepMode::kMergeOnly;
   const bool merge = a.mode != StepMode::kHeadOnly;
-  if (!a.step_idx || !a.workspace || !aligned16(a.workspace)) return DG_ERR_INVALID_ARG;
+  if (!a.step_idx) return DG_ERR_INVALID_ARG;
   if (head && (!a.h || !a.E || !aligned16(a.h) || !aligned16(a.E))) return DG_ERR_INVALID_ARG;
   if (merge && (!a.has_prev || !a.canvas || !a.prev_argmax || !a.accept || !a.entropy || !a.sampled ||
                 !a.argmax || !a.stop))
@@ -161,6 +165,18 @@ dg_status run_step(const StepArgs& a) {
   for (int b = 0; b < s.B; ++b)
     if (a.step_idx[b] < 0 || a.step_idx[b] >= pr.max_steps) return DG_ERR_RANGE;
   if (device_sms() <= 0) return DG_ERR_NO_DEVICE;
+  return DG_OK;
+}
+
+dg_status run_step(const StepArgs& a) {
+  dg_status st = check_step_inputs(a);
+  if (st != DG_OK) return st;
+  if (!a.workspace || !aligned16(a.workspace)) return DG_ERR_INVALID_ARG;
+  const dg_shape& s = *a.shape;
+  const dg_params& pr = *a.params;
+  const bool head = a.mode != StepMode::kMergeOnly;
+  const bool merge = a.mode != StepMode::kHeadOnly;
+  const bool fp8 = s.e_dtype == DG_E_FP8_E4M3;
   const int pairs = head_max_pairs(fp8);
   if (pairs <= 0) {
     snprintf(t_last_error, sizeof(t_last_error), "no CTA pair of the head kernel fits on this device");
@@ -175,15 +191,21 @@ dg_status run_step(const StepArgs& a) {
 
   CanvasParam cps[DG_MAX_B];
   memset(cps, 0, sizeof(cps));
+  uint8_t upd[DG_MAX_B] = {};  // the canvases this call updates, in order
+  int n_upd = 0;
   for (int b = 0; b < s.B; ++b) {
-    cps[b].k = a.step_idx[b];
+    // the kernels use k only as the Philox counter's step word
+    cps[b].k = static_cast<int32_t>(static_cast<uint32_t>(a.step_idx[b]) | (static_cast<uint32_t>(pr.block) << 16));
     cps[b].inv_tau = inv_tau_of(pr, a.step_idx[b]);
     cps[b].has_prev = (merge && a.has_prev[b]) ? 1 : 0;
     cps[b].active = (a.active == nullptr || a.active[b]) ? 1 : 0;
+    if (cps[b].active) upd[n_upd++] = static_cast<uint8_t>(b);
   }
+  if (n_upd == 0) return DG_OK;  // every canvas frozen: nothing to do
   const uint32_t seed_lo = static_cast<uint32_t>(pr.seed & 0xFFFFFFFFull);
   const uint32_t seed_hi = static_cast<uint32_t>(pr.seed >> 32);
   float* part = reinterpret_cast<float*>(wsb + ws.part_off);
+  int q_used = ws.P;  // records per row the head writes
 
   if (head) {
     // TMA boxes: one CTA's share of a stage, 128 rows x 128 bytes of K (the
@@ -230,7 +252,11 @@ dg_status run_step(const StepArgs& a) {
     hp.V = s.V;
     hp.B = s.B;
     hp.v_off = a.v_off;
-    hp.split = head_split(R, s.V, s.d, pairs, fp8 ? kBlockKFp8 : kBlockK);
+    // only the updated canvases' row tiles are split into work units; at
+    // most ws.P records per row (the workspace's planes)
+    hp.split = head_split(n_upd * s.L, s.V, s.d, pairs, fp8 ? kBlockKFp8 : kBlockK, ws.P);
+    memcpy(hp.mtile, upd, sizeof(upd));
+    q_used = hp.split.Q;
     hp.seed_lo = seed_lo;
     hp.seed_hi = seed_hi;
     // Philox4x32-10 round keys: key + i * (0x9E3779B9, 0xBB67AE85), mod 2^32
@@ -258,9 +284,9 @@ dg_status run_step(const StepArgs& a) {
   MergeParams mp;
   memset(&mp, 0, sizeof(mp));
   mp.R = R;
-  mp.B = s.B;
+  mp.B = n_upd;
   mp.V = s.V;
-  mp.P = a.mode == StepMode::kMergeOnly ? a.P : ws.P;
+  mp.P = a.mode == StepMode::kMergeOnly ? a.P : q_used;
   mp.S = a.mode == StepMode::kMergeOnly ? a.S : 1;
   mp.part = a.mode == StepMode::kMergeOnly ? a.part_in : part;
   mp.entropy = a.entropy;
@@ -279,11 +305,44 @@ dg_status run_step(const StepArgs& a) {
   mp.top_k = pr.top_k;
   mp.stop_entropy = pr.stop_entropy;
   memcpy(mp.cp, cps, sizeof(cps));
+  memcpy(mp.canvas_of, upd, sizeof(upd));
   if (!cuda_ok(launch_merge(mp, a.stream), "merge kernel launch")) return DG_ERR_CUDA;
   return DG_OK;
 }
 
 }  // namespace
+
+dg_status check_shape_and_params(const dg_shape* shape, const dg_params* params) {
+  const dg_status st = check_shape(shape);
+  return st != DG_OK ? st : check_params(params);
+}
+
+dg_status check_step_call(const dg_shape* shape, const dg_params* params, const void* h, const void* E,
+                          const float* e_scale, const int32_t* step_idx, const uint8_t* has_prev,
+                          int32_t* canvas, int32_t* prev_argmax, uint8_t* accept, float* entropy,
+                          int32_t* sampled, int32_t* argmax, int32_t* stop) {
+  StepArgs a{shape,   params,  h,      E,    e_scale, step_idx, has_prev, nullptr,  canvas, prev_argmax,
+             accept,  entropy, sampled, argmax, stop,   nullptr,  nullptr,  0, nullptr};
+  return check_step_inputs(a);
+}
+
+dg_status read_and_clear_latch(void* latch, cudaStream_t st) {
+  uint32_t err = 0;
+  if (!cuda_ok(cudaMemcpyAsync(&err, latch, sizeof(err), cudaMemcpyDeviceToHost, st), "fault latch read"))
+    return DG_ERR_CUDA;
+  if (!cuda_ok(cudaStreamSynchronize(st), "stream synchronise")) return DG_ERR_CUDA;
+  if (err != 0) {
+    if (!cuda_ok(cudaMemsetAsync(latch, 0, sizeof(err), st), "fault latch clear")) return DG_ERR_CUDA;
+    if (!cuda_ok(cudaStreamSynchronize(st), "stream synchronise")) return DG_ERR_CUDA;
+    if (err & ~static_cast<uint32_t>(kErrHiddenRange)) {
+      set_last_error_message("a device-side bounded wait ran out");
+      return DG_ERR_TIMEOUT;
+    }
+    set_last_error_message("FP8 head: a hidden-state value is not finite");
+    return DG_ERR_VALUE;
+  }
+  return DG_OK;
+}
 
 void set_last_error_message(const char* msg) {
   snprintf(t_last_error, sizeof(t_last_error), "%s", msg);
@@ -324,6 +383,7 @@ dg_params dg_default_params(void) {
   p.seed = 1234;
   p.selection_rule = DG_SELECT_CUMSUM;
   p.top_k = 1;
+  p.block = 0;
   return p;
 }
 
@@ -383,19 +443,7 @@ dg_status dg_debug_logits(const dg_shape* shape, const dg_params* params, const 
 
 dg_status dg_device_status(void* workspace, size_t ws_bytes, void* stream) {
   if (workspace == nullptr || ws_bytes < kAlign) return DG_ERR_INVALID_ARG;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint32_t err = 0;
-  if (cudaMemcpyAsync(&err, workspace, sizeof(err), cudaMemcpyDeviceToHost, st) != cudaSuccess)
-    return DG_ERR_CUDA;
-  if (cudaStreamSynchronize(st) != cudaSuccess) return DG_ERR_CUDA;
-  if (err != 0) {
-    if (cudaMemsetAsync(workspace, 0, sizeof(err), st) != cudaSuccess) return DG_ERR_CUDA;
-    if (cudaStreamSynchronize(st) != cudaSuccess) return DG_ERR_CUDA;
-    if (err & ~static_cast<uint32_t>(kErrHiddenRange)) return DG_ERR_TIMEOUT;
-    set_last_error_message("FP8 head: a hidden-state value is not finite");
-    return DG_ERR_VALUE;
-  }
-  return DG_OK;
+  return read_and_clear_latch(workspace, static_cast<cudaStream_t>(stream));
 }
 
 dg_status dg_denoise_loop(const dg_shape* shape, const dg_params* params, const void* E,

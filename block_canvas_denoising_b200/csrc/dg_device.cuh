@@ -318,13 +318,80 @@ DG_DEV void philox4x32_10_keys(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x
   out[3] = x3;
 }
 
+// Philox4x32-10 words of counter (x0, c1, c2, c3) for many x0 with c1..c3
+// fixed (one canvas slot at one step): the first round's product M1 c2 and
+// the second round's product M0 (hi(M1 c2) ^ c1 ^ k0) do not depend on x0,
+// so they are formed once per slot.  The outputs are those of
+// philox4x32_10_keys bit for bit.
+struct PhiloxRow {
+  uint32_t x0r1;  // word 0 after round 1:  hi(M1 c2) ^ c1 ^ k0[0]
+  uint32_t b1;    // lo(M1 c2) ^ k0[1]: round 2 mixes it into word 0
+  uint32_t e0;    // c3 ^ k1[0]: round 1 mixes it into word 2
+  uint32_t c1k;   // hi(M0 x0r1) ^ k1[1]: round 2 mixes it into word 2
+  uint32_t d;     // lo(M0 x0r1): word 3 after round 2
+};
+
+__host__ __device__ __forceinline__ PhiloxRow philox_row(uint32_t c1, uint32_t c2, uint32_t c3,
+                                                         const uint32_t (&k0)[10], const uint32_t (&k1)[10]) {
+  PhiloxRow r;
+  const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * c2;
+  r.x0r1 = static_cast<uint32_t>(p1 >> 32) ^ c1 ^ k0[0];
+  r.b1 = static_cast<uint32_t>(p1) ^ k0[1];
+  r.e0 = c3 ^ k1[0];
+  const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * r.x0r1;
+  r.c1k = static_cast<uint32_t>(p0 >> 32) ^ k1[1];
+  r.d = static_cast<uint32_t>(p0);
+  return r;
+}
+
+__host__ __device__ __forceinline__ void philox4x32_10_row(uint32_t x0, const PhiloxRow& r,
+                                                           const uint32_t (&k0)[10], const uint32_t (&k1)[10],
+                                                           uint32_t (&out)[4]) {
+  // round 1: only the product M0 x0 depends on x0
+  const uint64_t q0 = static_cast<uint64_t>(0xD2511F53u) * x0;
+  const uint32_t y2 = static_cast<uint32_t>(q0 >> 32) ^ r.e0;
+  const uint32_t x3a = static_cast<uint32_t>(q0);
+  // round 2: the product M0 x0r1 is the row's
+  const uint64_t q1 = static_cast<uint64_t>(0xCD9E8D57u) * y2;
+  uint32_t w0 = static_cast<uint32_t>(q1 >> 32) ^ r.b1;
+  uint32_t w1 = static_cast<uint32_t>(q1);
+  uint32_t w2 = r.c1k ^ x3a;
+  uint32_t w3 = r.d;
+#pragma unroll
+  for (int i = 2; i < 10; ++i) {
+    const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * w0;
+    const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * w2;
+    const uint32_t y0 = static_cast<uint32_t>(p1 >> 32) ^ w1 ^ k0[i];
+    const uint32_t y2b = static_cast<uint32_t>(p0 >> 32) ^ w3 ^ k1[i];
+    w1 = static_cast<uint32_t>(p1);
+    w3 = static_cast<uint32_t>(p0);
+    w0 = y0;
+    w2 = y2b;
+  }
+  out[0] = w0;
+  out[1] = w1;
+  out[2] = w2;
+  out[3] = w3;
+}
+
 // ---------------------------------------------------------------------------
-// Per-row partial of the fused head: base-2 online softmax of x = z / tau
-// (m2 = max x log2 e, S = sum 2^(x log2 e - m2), T2 = sum (x log2 e - m2)
-// 2^(...)), argmax of z, best specified Gumbel key.
+// Per-row partial of the fused head: base-2 online softmax of x = z / tau,
+// argmax of z, best specified Gumbel key.
+//
+// The softmax part is kept relative to the running maximum: m2 = fl(zmax c2)
+// (c2 = log2(e) / tau), every element other than the maximum contributes
+// e = 2^d with d = z c2 - m2 (one rounding), and the maximum itself is the
+// unit 2^0 -- it enters neither sum.  The record holds
+//   Sp = S - 1 = (number of elements equal to zmax) - 1 + sum_{z < zmax} e,
+//   T2 = sum_{z < zmax} d e,
+// so the normaliser's excess over the unit is carried explicitly and keeps
+// its relative precision however small it is (for a confident slot S - 1 is
+// far below the float32 spacing of S = 1).  The entropy follows as
+//   H = ln S - ln2 T2 / S = log1p(Sp) - ln2 T2 / (1 + Sp).
+// An empty record is m2 = -1e30, Sp = -1 (S = 0), T2 = 0.
 // ---------------------------------------------------------------------------
 struct Partial {
-  float m2, S, T2;
+  float m2, Sp, T2;
   float zmax;
   int zarg;
   float gkey;
@@ -333,7 +400,7 @@ struct Partial {
 
 DG_DEV void partial_init(Partial& a) {
   a.m2 = -1.0e30f;
-  a.S = 0.f;
+  a.Sp = -1.f;
   a.T2 = 0.f;
   a.zmax = -3.402823466e38f;
   a.zarg = 0x7fffffff;
@@ -341,16 +408,22 @@ DG_DEV void partial_init(Partial& a) {
   a.garg = 0x7fffffff;
 }
 
-// Merge b into a.  Softmax: m = max(m_a, m_b), S = sum_i S_i 2^(m_i - m),
-// T2 = sum_i (T2_i + (m_i - m) S_i) 2^(m_i - m).  Argmax and Gumbel key: the
+// Merge b into a.  Softmax: the record with the larger m2 keeps its unit;
+// the other's whole mass 1 + Sp_l moves into the ordinary mass, shifted by
+// dl = m2_l - m2_h <= 0:  Sp = Sp_h + (1 + Sp_l) 2^dl,
+// T2 = T2_h + (T2_l + dl (1 + Sp_l)) 2^dl.  Argmax and Gumbel key: the
 // larger value wins, ties to the lower vocabulary index.
 DG_DEV void partial_merge(Partial& a, const Partial& b) {
-  const float m = fmaxf(a.m2, b.m2);
-  const float da = a.m2 - m, db = b.m2 - m;
-  const float sa = exp2f(da), sb = exp2f(db);
-  a.T2 = (a.T2 + da * a.S) * sa + (b.T2 + db * b.S) * sb;
-  a.S = a.S * sa + b.S * sb;
-  a.m2 = m;
+  const bool bhi = b.m2 > a.m2;
+  const float mh = bhi ? b.m2 : a.m2, ml = bhi ? a.m2 : b.m2;
+  const float sph = bhi ? b.Sp : a.Sp, spl = bhi ? a.Sp : b.Sp;
+  const float th = bhi ? b.T2 : a.T2, tl = bhi ? a.T2 : b.T2;
+  const float dl = ml - mh;
+  const float sl = exp2f(dl);
+  const float tot_l = 1.0f + spl;
+  a.T2 = th + (tl + dl * tot_l) * sl;
+  a.Sp = fmaf(tot_l, sl, sph);
+  a.m2 = mh;
   if (b.zmax > a.zmax || (b.zmax == a.zmax && b.zarg < a.zarg)) {
     a.zmax = b.zmax;
     a.zarg = b.zarg;
@@ -364,6 +437,7 @@ DG_DEV void partial_merge(Partial& a, const Partial& b) {
 // Stream purposes (high half of counter word 1).
 constexpr uint32_t kPurposeGumbel = 0u;
 constexpr uint32_t kPurposeRenoise = 1u;
+constexpr uint32_t kPurposeInit = 3u;  // the noise canvas a block starts from
 
 // ---------------------------------------------------------------------------
 // The float32 key of the Gumbel-max draw, IEEE operations only.

@@ -59,17 +59,19 @@ constexpr uint64_t kDefaultWaitNs = 4000000000ull;
 
 // Per-canvas step data, filled on the host.
 struct CanvasParam {
-  int32_t k;        // step index
+  int32_t k;        // Philox counter step word: step index | block << 16
   float inv_tau;    // float32(1 / tau_k), tau_k in float64
   uint8_t has_prev;
   uint8_t active;
   uint8_t pad[2];
 };
 
-// Work split of the head: MT pair row tiles (256 rows) x NT vocabulary
-// tiles, cut into units of consecutive vocabulary tiles of one row tile.
-// Unit u covers row tile u % MT and vocabulary tiles [q NT / Q, (q+1) NT / Q),
-// q = u / MT; pair p runs units p, p + pairs, ...  grid = 2 * pairs CTAs.
+// Work split of the head: MT pair row tiles (256 rows, one canvas each) x NT
+// vocabulary tiles, cut into units of consecutive vocabulary tiles of one
+// row tile.  Unit u covers row tile u % MT and vocabulary tiles
+// [q NT / Q, (q+1) NT / Q), q = u / MT; pair p runs units p, p + pairs, ...
+// grid = 2 * pairs CTAs.  Row tile m is canvas HeadParams::mtile[m]: only
+// the canvases a step updates are split (a frozen canvas costs no work).
 struct HeadSplit {
   int MT, NT, KB, Q, units, pairs, grid;
 };
@@ -88,10 +90,13 @@ struct HeadParams {
   uint64_t wait_ns;
   uint32_t rk0[10], rk1[10];  // Philox round keys of the seed
   CanvasParam cp[DG_MAX_B];
+  uint8_t mtile[DG_MAX_B];     // canvas of row tile m (m < split.MT)
 };
 
 struct MergeParams {
-  int32_t R, B, V, P;
+  int32_t R;             // rows of the whole batch (plane stride of the records)
+  int32_t B;             // canvases this launch updates (canvas_of[0 .. B-1])
+  int32_t V, P;
   int32_t S;             // shards: records of row r are shard s's [7][R][P] block, s < S
   const float* part;
   float* entropy;
@@ -109,11 +114,13 @@ struct MergeParams {
   int32_t selection_rule;  // dg_selection
   int32_t top_k;
   CanvasParam cp[DG_MAX_B];
+  uint8_t canvas_of[DG_MAX_B];  // canvas of block group g (32 CTAs per canvas)
 };
 
 // kblock: K elements per stage (kBlockK, or kBlockKFp8 for the FP8 head);
-// KB = ceil(d / kblock), the last stage's K tail read as zeros.
-HeadSplit head_split(int R, int V, int d, int max_pairs, int kblock);
+// KB = ceil(d / kblock), the last stage's K tail read as zeros.  At most
+// q_cap units per row tile (the records per row the workspace holds).
+HeadSplit head_split(int R, int V, int d, int max_pairs, int kblock, int q_cap = 1 << 30);
 int head_max_pairs(bool fp8);
 
 // Workspace layout (byte offsets), see dg_workspace_size().
@@ -129,6 +136,19 @@ WsLayout ws_layout(const dg_shape& s, int max_pairs);
 // Text returned by dg_last_error_message() on this host thread.
 void set_last_error_message(const char* msg);
 
+// The argument checks of dg_denoise_step other than those of the workspace
+// (shape, parameters, pointers, alignment, step range, device): DG_OK or
+// the status dg_denoise_step would return, before anything is enqueued.
+dg_status check_step_call(const dg_shape* shape, const dg_params* params, const void* h, const void* E,
+                          const float* e_scale, const int32_t* step_idx, const uint8_t* has_prev,
+                          int32_t* canvas, int32_t* prev_argmax, uint8_t* accept, float* entropy,
+                          int32_t* sampled, int32_t* argmax, int32_t* stop);
+
+// Synchronise `st`, read the 32-bit fault latch at `latch` (device), clear it
+// if set, and map it to a status (DG_OK, DG_ERR_TIMEOUT, DG_ERR_VALUE,
+// DG_ERR_CUDA).
+dg_status read_and_clear_latch(void* latch, cudaStream_t st);
+
 // bf16 head: tmA = h bf16 [R, d], tmB = E bf16 [V, d] (tmA2 unused).
 // FP8 head:  tmA = h1, tmA2 = h2 (E4M3 [R, d]), tmB = E codes E4M3 [V, d].
 cudaError_t launch_head(bool fp8, const CUtensorMap& tmA, const CUtensorMap& tmA2, const CUtensorMap& tmB,
@@ -139,6 +159,12 @@ cudaError_t launch_head(bool fp8, const CUtensorMap& tmA, const CUtensorMap& tmA
 cudaError_t launch_hidden_split(const void* h, uint8_t* h1, uint8_t* h2, float* rinv, int R, int d,
                                 uint32_t* err, cudaStream_t stream);
 cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream);
+// canvas[b * L + s] = (r V) >> 32, r = Philox word 0 of counter
+// (0, s | 3 << 16, ctr_step, b): the uniform noise a block starts from.
+cudaError_t launch_init_canvas(int32_t* canvas, int B, int L, int V, uint32_t ctr_step, uint32_t seed_lo,
+                               uint32_t seed_hi, cudaStream_t stream);
+// The argument checks shared by the entry points (shape; parameters).
+dg_status check_shape_and_params(const dg_shape* shape, const dg_params* params);
 cudaError_t launch_wait_selftest(uint32_t* err, uint64_t limit_ns, cudaStream_t stream);
 cudaError_t launch_gumbel_probe(const uint32_t* words, int n, float* g_exact, float* lg2e_approx,
                                 cudaStream_t stream);

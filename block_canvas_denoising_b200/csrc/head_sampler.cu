@@ -6,7 +6,8 @@
 // each 128 x 256 float32 accumulator tile lives in tensor memory (TMEM) and
 // is reduced in place by the epilogue warps into per-row partials of
 //   * the online softmax of x = z / tau_k in base 2: m2 = max x log2(e),
-//     S = sum 2^(x log2 e - m2), T2 = sum (x log2 e - m2) 2^(...)  -- the
+//     S = sum 2^(x log2 e - m2), T2 = sum (x log2 e - m2) 2^(...), carried
+//     as Sp = S - 1 with the maximum's unit mass kept out of the sums -- the
 //     entropy of the tempered distribution follows as ln S - ln2 T2 / S
 //     ([Docs] "DiffusionGemma", Recommended serving configuration: entropy
 //     drives token selection and adaptive stopping; temperature schedule);
@@ -42,14 +43,18 @@
 
 #include "dg_device.cuh"
 #include "dg_internal.h"
+#include "per_device.h"
 
 namespace dg {
 
 namespace {
 
-DG_DEV void unit_range(const HeadSplit& sp, int u, int& m, int& n0, int& n1, int& q) {
+// Unit u: row tile (canvas) m, vocabulary tiles [n0, n1), unit index q
+// within the row tile.
+DG_DEV void unit_range(const HeadParams& p, int u, int& m, int& n0, int& n1, int& q) {
+  const HeadSplit& sp = p.split;
   q = u / sp.MT;
-  m = u - q * sp.MT;
+  m = p.mtile[u - q * sp.MT];
   n0 = static_cast<int>((static_cast<int64_t>(q) * sp.NT) / sp.Q);
   n1 = static_cast<int>((static_cast<int64_t>(q + 1) * sp.NT) / sp.Q);
 }
@@ -108,12 +113,13 @@ DG_DEV void top2(float& a1, float& a2, float b1, float b2) {
   a1 = hi;
 }
 
-// The Philox words of the 8 consecutive vocabulary entries 4 cb .. 4 cb + 7.
-DG_DEV void philox_words8(uint32_t cb, uint32_t ctr1, uint32_t ctr2, uint32_t ctr3, const uint32_t (&rk0)[10],
-                          const uint32_t (&rk1)[10], uint32_t (&w)[8]) {
+// The Philox words of the 8 consecutive vocabulary entries 4 cb .. 4 cb + 7
+// of the slot whose row constants are `pr`.
+DG_DEV void philox_words8(uint32_t cb, const PhiloxRow& pr, const uint32_t (&rk0)[10], const uint32_t (&rk1)[10],
+                          uint32_t (&w)[8]) {
   uint32_t wa[4], wb[4];
-  philox4x32_10_keys(cb, ctr1, ctr2, ctr3, rk0, rk1, wa);
-  philox4x32_10_keys(cb + 1, ctr1, ctr2, ctr3, rk0, rk1, wb);
+  philox4x32_10_row(cb, pr, rk0, rk1, wa);
+  philox4x32_10_row(cb + 1, pr, rk0, rk1, wb);
 #pragma unroll
   for (int l = 0; l < 4; ++l) {
     w[l] = wa[l];
@@ -127,46 +133,61 @@ DG_DEV void philox_words8(uint32_t cb, uint32_t ctr1, uint32_t ctr2, uint32_t ct
 // wm_pre: when have_wm (warp-uniform), the group's largest Philox word,
 // computed beforehand by another warp; the words themselves are then drawn
 // here only if the group passes its bound.
-DG_DEV void process8(const float (&z)[8], int v0, float inv_tau, float c2, uint32_t ctr1,
-                     uint32_t ctr2, uint32_t ctr3, const uint32_t (&rk0)[10], const uint32_t (&rk1)[10],
-                     float thr, bool have_wm, uint32_t wm_pre, Partial& pt, Screen& sc) {
-  // ---- group max, argmax of z (ties to the lower index; groups arrive in
-  // increasing v)
+DG_DEV void process8(const float (&z)[8], int v0, float inv_tau, float c2, const PhiloxRow& pr,
+                     const uint32_t (&rk0)[10], const uint32_t (&rk1)[10], float thr, bool have_wm,
+                     uint32_t wm_pre, Partial& pt, Screen& sc) {
+  // ---- group max; does the group hold the row's running maximum?  (c2 > 0,
+  // so the maximum of z is the maximum of x; groups arrive in increasing v)
   const float m01 = fmaxf(z[0], z[1]), m23 = fmaxf(z[2], z[3]);
   const float m45 = fmaxf(z[4], z[5]), m67 = fmaxf(z[6], z[7]);
   const float gmax = fmaxf(fmaxf(m01, m23), fmaxf(m45, m67));
-  if (gmax > pt.zmax) {
+  if (gmax >= pt.zmax) {
+    // elements equal to the maximum are units (exponent exactly 0): count
+    // them, and find the first (the argmax, ties to the lower index)
+    float neq = 0.f;
     int jj = 7;
 #pragma unroll
-    for (int j = 6; j >= 0; --j) jj = (z[j] == gmax) ? j : jj;
-    pt.zmax = gmax;
-    pt.zarg = v0 + jj;
+    for (int j = 7; j >= 0; --j) {
+      const bool eq = z[j] == gmax;
+      neq += eq ? 1.f : 0.f;
+      jj = eq ? j : jj;
+    }
+    if (gmax > pt.zmax) {
+      // new maximum: the old total mass 1 + Sp joins the ordinary mass,
+      // shifted by delta = m2_old - m2_new <= 0
+      const float nm2 = gmax * c2;
+      const float delta = pt.m2 - nm2;
+      const float scl = ex2_approx(delta);
+      const float tot = 1.0f + pt.Sp;
+      pt.T2 = (pt.T2 + delta * tot) * scl;
+      pt.Sp = fmaf(tot, scl, neq - 1.0f);
+      pt.m2 = nm2;
+      pt.zmax = gmax;
+      pt.zarg = v0 + jj;
+    } else {
+      pt.Sp += neq;  // exact ties with the running maximum: more units
+    }
   }
 
-  // ---- online softmax partial, base 2
-  const float gm2 = gmax * c2;
-  if (gm2 > pt.m2) {
-    const float delta = pt.m2 - gm2;
-    const float scl = ex2_approx(delta);
-    pt.T2 = (pt.T2 + delta * pt.S) * scl;
-    pt.S = pt.S * scl;
-    pt.m2 = gm2;
-  }
+  // ---- online softmax partial, base 2: every element below the maximum
   {
     const float nm = -pt.m2;
+    const float zm = pt.zmax;
     float s0 = 0.f, s1 = 0.f, t0 = 0.f, t1 = 0.f;
 #pragma unroll
     for (int j = 0; j < 8; j += 2) {
       const float d0 = fmaf(z[j], c2, nm);
       const float d1 = fmaf(z[j + 1], c2, nm);
-      const float e0 = ex2_approx(d0);
-      const float e1 = ex2_approx(d1);
+      const float x0 = ex2_approx(d0);
+      const float x1 = ex2_approx(d1);
+      const float e0 = z[j] < zm ? x0 : 0.f;
+      const float e1 = z[j + 1] < zm ? x1 : 0.f;
       s0 += e0;
       s1 += e1;
       t0 = fmaf(d0, e0, t0);
       t1 = fmaf(d1, e1, t1);
     }
-    pt.S += s0 + s1;
+    pt.Sp += s0 + s1;
     pt.T2 += t0 + t1;
   }
 
@@ -185,9 +206,9 @@ DG_DEV void process8(const float (&z)[8], int v0, float inv_tau, float c2, uint3
   uint32_t w[8];
   if (have_wm) {
     if (__fmaf_rn(lg2_exp1_approx(wm_pre), -kLn2, x0max) < lim_eps) return;
-    philox_words8(cb, ctr1, ctr2, ctr3, rk0, rk1, w);
+    philox_words8(cb, pr, rk0, rk1, w);
   } else {
-    philox_words8(cb, ctr1, ctr2, ctr3, rk0, rk1, w);
+    philox_words8(cb, pr, rk0, rk1, w);
     const uint32_t wm = max(max(max(w[0], w[1]), max(w[2], w[3])), max(max(w[4], w[5]), max(w[6], w[7])));
     if (__fmaf_rn(lg2_exp1_approx(wm), -kLn2, x0max) < lim_eps) return;
   }
@@ -233,8 +254,8 @@ DG_DEV void process8(const float (&z)[8], int v0, float inv_tau, float c2, uint3
 // logits dump, then the group's reductions.
 template <bool kFp8>
 DG_DEV void epi_group(const uint32_t* r, int v0, int row, float rinv, float inv_tau, float c2,
-                      uint32_t ctr1, uint32_t ctr2, uint32_t ctr3, float thr, bool have_wm, uint32_t wm_pre,
-                      const HeadParams& p, Partial& pt, Screen& sc) {
+                      const PhiloxRow& pr, float thr, bool have_wm, uint32_t wm_pre, const HeadParams& p,
+                      Partial& pt, Screen& sc) {
   float z[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) z[j] = __uint_as_float(r[j]);
@@ -252,7 +273,7 @@ DG_DEV void epi_group(const uint32_t* r, int v0, int row, float rinv, float inv_
   }
   // z, e_scale and the dump are indexed within this launch's rows of E; the
   // sampler (Philox counters, token indices) uses the global vocabulary index
-  process8(z, v0 + p.v_off, inv_tau, c2, ctr1, ctr2, ctr3, p.rk0, p.rk1, thr, have_wm, wm_pre, pt, sc);
+  process8(z, v0 + p.v_off, inv_tau, c2, pr, p.rk0, p.rk1, thr, have_wm, wm_pre, pt, sc);
 }
 
 // Named barrier over the epilogue warps only (barrier 1).
@@ -339,7 +360,7 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       bool ok = true;
       for (int u = pair; u < sp.units && ok; u += npairs) {
         int m, n0, n1, q;
-        unit_range(sp, u, m, n0, n1, q);
+        unit_range(p, u, m, n0, n1, q);
         for (int n = n0; n < n1 && ok; ++n) {
           for (int kb = 0; kb < sp.KB; ++kb) {
             if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, p.wait_ns)) {
@@ -398,7 +419,7 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       bool ok = true;
       for (int u = pair; u < sp.units && ok; u += npairs) {
         int m, n0, n1, q;
-        unit_range(sp, u, m, n0, n1, q);
+        unit_range(p, u, m, n0, n1, q);
         for (int n = n0; n < n1 && ok; ++n, ++tile) {
           const int acc = tile & 1;
           const uint32_t acc_phase = (tile >> 1) & 1;
@@ -473,9 +494,9 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         const int hrow = m_t * kPairM + static_cast<int>(rank) * kBlockM + kMmaQuarter * 32 + r;
         const int hb = hrow >> 8;
         uint32_t w[8];
-        philox_words8(static_cast<uint32_t>(p.v_off + n_t * kBlockN + g * 8) >> 2,
-                      static_cast<uint32_t>(hrow & 255) | (kPurposeGumbel << 16), static_cast<uint32_t>(p.cp[hb].k),
-                      static_cast<uint32_t>(hb), p.rk0, p.rk1, w);
+        const PhiloxRow pr = philox_row(static_cast<uint32_t>(hrow & 255) | (kPurposeGumbel << 16),
+                                        static_cast<uint32_t>(p.cp[hb].k), static_cast<uint32_t>(hb), p.rk0, p.rk1);
+        philox_words8(static_cast<uint32_t>(p.v_off + n_t * kBlockN + g * 8) >> 2, pr, p.rk0, p.rk1, w);
         dst[g * 32 + r] = max(max(max(w[0], w[1]), max(w[2], w[3])), max(max(w[4], w[5]), max(w[6], w[7])));
       }
       __syncwarp();
@@ -488,12 +509,12 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     bool ok = true;
     if (!mma_quarter) {
       int m, n0, n1, q;
-      unit_range(sp, pair, m, n0, n1, q);
+      unit_range(p, pair, m, n0, n1, q);
       ok = produce_words(0, m, n0);
     }
     for (int u = pair; u < sp.units; u += npairs) {
       int m, n0, n1, q;
-      unit_range(sp, u, m, n0, n1, q);
+      unit_range(p, u, m, n0, n1, q);
       const int row = m * kPairM + static_cast<int>(rank) * kBlockM + rloc;
       const int b = row >> 8;
       const int slot = row & 255;
@@ -501,9 +522,9 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       const float inv_tau = cp.inv_tau;
       const float rinv = kFp8 ? __ldg(p.row_inv + row) : 1.0f;
       const float c2 = __fmul_rn(inv_tau, kLog2e);
-      const uint32_t ctr1 = static_cast<uint32_t>(slot) | (kPurposeGumbel << 16);
-      const uint32_t ctr2 = static_cast<uint32_t>(cp.k);
-      const uint32_t ctr3 = static_cast<uint32_t>(b);
+      // Philox counter (v >> 2, slot | purpose << 16, k, b): the row's constants
+      const PhiloxRow pr = philox_row(static_cast<uint32_t>(slot) | (kPurposeGumbel << 16),
+                                      static_cast<uint32_t>(cp.k), static_cast<uint32_t>(b), p.rk0, p.rk1);
       Partial pt;
       partial_init(pt);
       Screen sc;
@@ -521,7 +542,7 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           bool more = nn < n1;
           if (!more && u + npairs < sp.units) {
             int n1n, qn;
-            unit_range(sp, u + npairs, mn, nn, n1n, qn);
+            unit_range(p, u + npairs, mn, nn, n1n, qn);
             more = true;
           }
           if (more && !produce_words(tile + 1, mn, nn)) {
@@ -562,11 +583,11 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 #pragma unroll 1
         for (int g = 0; g < kGroups; g += 2) {
           tmem_load8_issue(tbase + 8 * (g + 1), rb);
-          epi_group<kFp8>(ra, vbase + 8 * g, row, rinv, inv_tau, c2, ctr1, ctr2, ctr3, thr, mma_quarter,
+          epi_group<kFp8>(ra, vbase + 8 * g, row, rinv, inv_tau, c2, pr, thr, mma_quarter,
                           mma_quarter ? wsrc[g * 32] : 0u, p, pt, sc);
           tmem_load8_wait(rb);
           if (g + 2 < kGroups) tmem_load8_issue(tbase + 8 * (g + 2), ra);
-          epi_group<kFp8>(rb, vbase + 8 * (g + 1), row, rinv, inv_tau, c2, ctr1, ctr2, ctr3, thr, mma_quarter,
+          epi_group<kFp8>(rb, vbase + 8 * (g + 1), row, rinv, inv_tau, c2, pr, thr, mma_quarter,
                           mma_quarter ? wsrc[(g + 1) * 32] : 0u, p, pt, sc);
           tmem_load8_wait(ra);
           __syncwarp();
@@ -592,7 +613,7 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       if (cg != 0) {
         float* d = sPart + (cg * kPartialFields) * kBlockM + rloc;
         d[0 * kBlockM] = pt.m2;
-        d[1 * kBlockM] = pt.S;
+        d[1 * kBlockM] = pt.Sp;
         d[2 * kBlockM] = pt.T2;
         d[3 * kBlockM] = pt.zmax;
         d[4 * kBlockM] = __int_as_float(pt.zarg);
@@ -606,7 +627,7 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           const float* s2 = sPart + (g2 * kPartialFields) * kBlockM + rloc;
           Partial o;
           o.m2 = s2[0 * kBlockM];
-          o.S = s2[1 * kBlockM];
+          o.Sp = s2[1 * kBlockM];
           o.T2 = s2[2 * kBlockM];
           o.zmax = s2[3 * kBlockM];
           o.zarg = __float_as_int(s2[4 * kBlockM]);
@@ -618,7 +639,7 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         const size_t idx = static_cast<size_t>(row) * sp.Q + q;
         float* part = p.part;
         part[0 * plane + idx] = pt.m2;
-        part[1 * plane + idx] = pt.S;
+        part[1 * plane + idx] = pt.Sp;
         part[2 * plane + idx] = pt.T2;
         part[3 * plane + idx] = pt.zmax;
         part[4 * plane + idx] = __int_as_float(pt.zarg);
@@ -647,13 +668,14 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   }
 }
 
+// Launch set-up of one head variant on the current device: allow its
+// dynamic shared memory, then count the CTA pairs that fit at once.
 template <bool kFp8>
-int max_pairs_of() {
-  static int cached = -1;
-  if (cached > 0) return cached;
+bool setup_on_current_device(int* pairs) {
   constexpr int kSmem = HeadCfg<kFp8>::kSmemBytes;
-  cudaError_t e = cudaFuncSetAttribute(head_sampler_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-  if (e != cudaSuccess) return -1;
+  if (cudaFuncSetAttribute(head_sampler_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) !=
+      cudaSuccess)
+    return false;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2, 1, 1);
   cfg.blockDim = dim3(kHeadThreads, 1, 1);
@@ -666,14 +688,25 @@ int max_pairs_of() {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, head_sampler_kernel<kFp8>, &cfg) != cudaSuccess || n < 1) return -1;
-  cached = n;
-  return cached;
+  if (cudaOccupancyMaxActiveClusters(&n, head_sampler_kernel<kFp8>, &cfg) != cudaSuccess || n < 1) return false;
+  *pairs = n;
+  return true;
+}
+
+// Co-resident CTA pairs of a head variant on the current device (-1 if it
+// cannot run there), set up once per device.
+template <bool kFp8>
+int max_pairs_of() {
+  static PerDevice<int> cache;
+  int dev = -1, pairs = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (!cache.get(dev, [](int* v) { return setup_on_current_device<kFp8>(v); }, &pairs)) return -1;
+  return pairs;
 }
 
 int head_max_pairs(bool fp8) { return fp8 ? max_pairs_of<true>() : max_pairs_of<false>(); }
 
-HeadSplit head_split(int R, int V, int d, int max_pairs, int kblock) {
+HeadSplit head_split(int R, int V, int d, int max_pairs, int kblock, int q_cap) {
   HeadSplit s;
   s.MT = R / kPairM;
   s.NT = V / kBlockN;
@@ -687,6 +720,7 @@ HeadSplit head_split(int R, int V, int d, int max_pairs, int kblock) {
     if (q > s.NT) q = s.NT;
     s.Q = q;  // about one unit per pair
   }
+  if (s.Q > q_cap) s.Q = q_cap;
   s.units = s.MT * s.Q;
   s.pairs = s.units < max_pairs ? s.units : max_pairs;
   s.grid = 2 * s.pairs;

@@ -32,7 +32,7 @@ constexpr int kRowsPerCta = 8;  // one warp per row
 DG_DEV Partial partial_load(const float* part, size_t plane, size_t idx) {
   Partial a;
   a.m2 = __ldcg(part + 0 * plane + idx);
-  a.S = __ldcg(part + 1 * plane + idx);
+  a.Sp = __ldcg(part + 1 * plane + idx);
   a.T2 = __ldcg(part + 2 * plane + idx);
   a.zmax = __ldcg(part + 3 * plane + idx);
   a.zarg = __float_as_int(__ldcg(part + 4 * plane + idx));
@@ -44,7 +44,7 @@ DG_DEV Partial partial_load(const float* part, size_t plane, size_t idx) {
 DG_DEV Partial partial_shfl_down(const Partial& a, int off) {
   Partial o;
   o.m2 = __shfl_down_sync(0xffffffffu, a.m2, off);
-  o.S = __shfl_down_sync(0xffffffffu, a.S, off);
+  o.Sp = __shfl_down_sync(0xffffffffu, a.Sp, off);
   o.T2 = __shfl_down_sync(0xffffffffu, a.T2, off);
   o.zmax = __shfl_down_sync(0xffffffffu, a.zmax, off);
   o.zarg = __shfl_down_sync(0xffffffffu, a.zarg, off);
@@ -65,7 +65,9 @@ merge_select_kernel(const __grid_constant__ MergeParams p) {
   const int t = threadIdx.x;
   const int warp = t >> 5;
   const int lane = t & 31;
-  const int row = blockIdx.x * kRowsPerCta + warp;
+  constexpr int kCtasPerCanvas = 256 / kRowsPerCta;
+  const int b = p.canvas_of[blockIdx.x / kCtasPerCanvas];  // only the canvases this step updates
+  const int row = b * 256 + (blockIdx.x % kCtasPerCanvas) * kRowsPerCta + warp;
   const size_t plane = static_cast<size_t>(p.R) * p.P;
 
   // Launched as a programmatic dependent of the head kernel: wait until its
@@ -88,22 +90,22 @@ merge_select_kernel(const __grid_constant__ MergeParams p) {
   }
   if (lane == 0) {
     p.row_rec[row] = 0u;  // the head's key record of this row starts empty next step
-    // H = ln S - ln2 T2 / S, clamped at 0 (the exact value is >= 0)
-    float H = logf(a.S) - kLn2 * a.T2 / a.S;
-    H = fmaxf(H, 0.0f);
-    p.entropy[row] = H;
+    // H = ln S - ln2 T2 / S with S = 1 + Sp, in float64 from the float32
+    // record, clamped at 0 (the exact value is >= 0)
+    const double sp = static_cast<double>(a.Sp);
+    double H = log1p(sp) - 0.69314718055994530942 * static_cast<double>(a.T2) / (1.0 + sp);
+    H = H > 0.0 ? H : 0.0;
+    p.entropy[row] = static_cast<float>(H);
     p.sampled[row] = a.garg;
     p.argmax[row] = a.zarg;
   }
 
   // ---- ticket: the last CTA of this canvas does the per-canvas step
-  const int b = (blockIdx.x * kRowsPerCta) >> 8;
   __threadfence();
   __syncthreads();
   if (t == 0) {
-    const uint32_t ctas_per_canvas = 256 / kRowsPerCta;
     const uint32_t prev = atomicAdd(&p.tickets[b], 1u);
-    s_last = (prev == ctas_per_canvas - 1) ? 1 : 0;
+    s_last = (prev == kCtasPerCanvas - 1) ? 1 : 0;
     if (s_last) p.tickets[b] = 0u;  // reset for the next step
   }
   __syncthreads();
@@ -162,7 +164,7 @@ merge_select_kernel(const __grid_constant__ MergeParams p) {
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) hsum += __shfl_xor_sync(0xffffffffu, hsum, off);
   if ((t & 31) == 0) s_red[t >> 5] = hsum;
-  const int prev = cp.active ? p.prev_argmax[grow] : amax;
+  const int prev = p.prev_argmax[grow];
   const int same = __syncthreads_and(prev == amax);
   double total = 0.0;
 #pragma unroll
@@ -170,17 +172,15 @@ merge_select_kernel(const __grid_constant__ MergeParams p) {
   const double mean_h = total / 256.0;
   const bool stop = cp.has_prev && same && (mean_h < p.stop_entropy);
 
-  if (cp.active) {
-    p.accept[grow] = accepted ? 1 : 0;
-    p.canvas[grow] = tok;
-    p.prev_argmax[grow] = amax;
-    if (t == 0) p.stop[b] = stop ? 1 : 0;
-  }
+  p.accept[grow] = accepted ? 1 : 0;
+  p.canvas[grow] = tok;
+  p.prev_argmax[grow] = amax;
+  if (t == 0) p.stop[b] = stop ? 1 : 0;
 }
 
 cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.R / kRowsPerCta, 1, 1);
+  cfg.gridDim = dim3(p.B * (256 / kRowsPerCta), 1, 1);  // p.B: canvases updated
   cfg.blockDim = dim3(256, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;

@@ -62,11 +62,17 @@ extern "C" dg_status dg_denoise_step_noalloc(const dg_shape* shape, const dg_par
                                              const uint8_t* has_prev, const uint8_t* active, int32_t* canvas,
                                              int32_t* prev_argmax, uint8_t* accept, float* entropy,
                                              int32_t* sampled, int32_t* argmax, int32_t* stop, void* stream) {
-  if (shape == nullptr) return DG_ERR_INVALID_ARG;
+  // Every argument check runs before anything touches the shared array.
+  dg_status st = dg::check_step_call(shape, params, h, E, e_scale, step_idx, has_prev, canvas, prev_argmax,
+                                     accept, entropy, sampled, argmax, stop);
+  if (st != DG_OK) return st;
   const size_t need = dg_workspace_size(shape);
-  if (need == 0) return DG_ERR_UNSUPPORTED_SHAPE;
+  if (need == 0) {
+    dg::set_last_error_message("dg_denoise_step_noalloc: the head kernel cannot run on this device");
+    return DG_ERR_CUDA;
+  }
   if (need > kNoAllocScratchBytes) {
-    char msg[160];
+    char msg[200];
     snprintf(msg, sizeof(msg),
              "dg_denoise_step_noalloc: this shape needs %zu bytes of scratch, the fixed array holds %zu",
              need, kNoAllocScratchBytes);
@@ -74,15 +80,39 @@ extern "C" dg_status dg_denoise_step_noalloc(const dg_shape* shape, const dg_par
     return DG_ERR_WORKSPACE;
   }
   void* ws = nullptr;
-  dg_status st = scratch_address(&ws);
-  if (st != DG_OK) return st;
-  // The array keeps the previous call's contents.  The fault latch, the
-  // per-canvas tickets and the per-row key records must start at zero
-  // (everything else is written before it is read), so clear them on the
-  // caller's stream; this does not allocate.
-  const size_t zero_bytes =
-      dg::ws_layout(*shape, dg::head_max_pairs(shape->e_dtype == DG_E_FP8_E4M3)).zero_prefix;
-  if (cudaMemsetAsync(ws, 0, zero_bytes, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DG_ERR_CUDA;
+  if ((st = scratch_address(&ws)) != DG_OK) return st;
+  // The array keeps the previous call's contents.  The per-canvas tickets
+  // and the per-row key records must start at zero (everything after them
+  // is written before it is read), so clear them on the caller's stream;
+  // this does not allocate.  The fault latch in front of them is left as it
+  // is: a fault of an earlier call stays there until dg_noalloc_status()
+  // reads and clears it.
+  const dg::WsLayout lay = dg::ws_layout(*shape, dg::head_max_pairs(shape->e_dtype == DG_E_FP8_E4M3));
+  const cudaError_t e = cudaMemsetAsync(static_cast<unsigned char*>(ws) + lay.tickets_off, 0,
+                                        lay.zero_prefix - lay.tickets_off, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    char msg[200];
+    snprintf(msg, sizeof(msg), "dg_denoise_step_noalloc: clearing the scratch array: %s", cudaGetErrorString(e));
+    dg::set_last_error_message(msg);
+    return DG_ERR_CUDA;
+  }
   return dg_denoise_step(shape, params, h, E, e_scale, step_idx, has_prev, active, canvas, prev_argmax, accept,
                          entropy, sampled, argmax, stop, ws, kNoAllocScratchBytes, stream);
+}
+
+extern "C" dg_status dg_noalloc_status(void* stream) {
+  void* ws = nullptr;
+  const dg_status st = scratch_address(&ws);
+  if (st != DG_OK) return st;
+  return dg::read_and_clear_latch(ws, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" dg_status dg_noalloc_selftest_bounded_wait(uint64_t limit_ns, void* stream) {
+  void* ws = nullptr;
+  const dg_status st = scratch_address(&ws);
+  if (st != DG_OK) return st;
+  if (dg::launch_wait_selftest(static_cast<uint32_t*>(ws), limit_ns, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return DG_ERR_CUDA;
+  return dg_noalloc_status(stream);
 }

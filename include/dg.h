@@ -87,7 +87,7 @@ typedef enum { DG_SELECT_CUMSUM = 0, DG_SELECT_MI = 1, DG_SELECT_TOPK = 2 } dg_s
 
 /* Sampler parameters; dg_default_params() gives the [Docs] serving
  * defaults (tau0 0.8, tau1 0.4, 48 steps, bound 0.1, stop 0.005,
- * DG_SELECT_CUMSUM). */
+ * DG_SELECT_CUMSUM, seed 1234, block 0). */
 typedef struct {
   double tau0;             /* temperature at step 0 */
   double tau1;             /* temperature at step max_steps-1 */
@@ -97,6 +97,12 @@ typedef struct {
   uint64_t seed;           /* Philox4x32-10 key (low word, high word) */
   int32_t selection_rule;  /* a dg_selection */
   int32_t top_k;           /* slots accepted by DG_SELECT_TOPK */
+  int32_t block;           /* index of the canvas block in a block-by-block
+                              generation (0 for a single block): every
+                              block draws its own random streams, the
+                              Philox counter's step word being
+                              k | block << 16 (0 <= block < 65536;
+                              max_steps <= 65536) */
 } dg_params;
 
 dg_params dg_default_params(void);
@@ -133,8 +139,10 @@ dg_status dg_workspace_init(void* workspace, size_t ws_bytes, void* stream);
  *             ([Docs] temperature schedule), tau0 for max_steps == 1.
  *   has_prev  HOST uint8 [B]: 1 if prev_argmax holds the previous step's
  *             prediction for that canvas (0 on a canvas's first step).
- *   active    HOST uint8 [B] or NULL (= all 1): canvases with 0 are left
- *             untouched (canvas, prev_argmax, accept, stop not written).
+ *   active    HOST uint8 [B] or NULL (= all 1): canvases with 0 are frozen:
+ *             they cost no head or merge work and none of their outputs
+ *             (canvas, prev_argmax, accept, entropy, sampled, argmax, stop)
+ *             is written.  With every canvas frozen nothing is launched.
  * In/out
  *   canvas      int32 [B*L]: overwritten with the new canvas (accepted slots
  *               take the sampled token, the rest a uniform random token).
@@ -196,7 +204,9 @@ typedef int (*dg_hidden_fn)(int32_t k, const int32_t* canvas, void* h_out,
  *   prev_argmax  int32 [B*L] in/out: prediction state (see has_prev).
  *   has_prev     HOST uint8 [B] in/out: resume state; all 0 for a fresh start.
  *   steps_taken  HOST int32 [B] out: steps run for each canvas.
- *   accept, entropy, sampled, argmax, stop: device outputs of the last step.
+ *   accept, entropy, sampled, argmax, stop: device outputs of each canvas's
+ *                last step (a frozen canvas is skipped by the later steps:
+ *                it costs no head work and its outputs are left as they were).
  * Resuming with the state of an interrupted loop at k_start gives the same
  * result as the uninterrupted run (the random streams are counter-based).
  */
@@ -209,6 +219,46 @@ dg_status dg_denoise_loop(const dg_shape* shape, const dg_params* params,
                           int32_t* argmax, int32_t* stop,
                           void* workspace, size_t ws_bytes, void* stream);
 
+/* ---- block-by-block generation ([Report] Figure 4: encode & append) ----
+ * Generation runs block after block: each block of B canvases starts from
+ * uniform noise, the adaptive loop denoises it until it settles, and the
+ * committed block is appended to the context the next block is conditioned
+ * on.  The model that encodes the committed blocks and produces the hidden
+ * states is the caller's (hidden_fn); this library runs the blocks' steps. */
+
+/* Fill canvas (int32 [B*L], device) with the uniform noise block
+ * params->block starts from ([Report] Figure 3: uniform noise): token
+ * (r V) >> 32 of Philox counter (0, slot | 3 << 16, block << 16, b), lane 0. */
+dg_status dg_init_canvas(const dg_shape* shape, const dg_params* params, int32_t* canvas, void* stream);
+
+/* Hidden-state producer of block j: writes the bf16 [B*L, d] hidden states
+ * of step k of block j into h_out (device) given the block's current canvas
+ * (device int32 [B*L]) and the blocks committed before it (device int32
+ * [j][B*L], the first j rows of dg_generate_blocks' `blocks`; NULL for
+ * j = 0), enqueued on `stream`.  Returns 0 on success; anything else stops
+ * the generation with DG_ERR_CALLBACK. */
+typedef int (*dg_block_hidden_fn)(int32_t block, int32_t k, const int32_t* canvas,
+                                  const int32_t* committed, void* h_out, void* user, void* stream);
+
+/* dg_generate_blocks -- n_blocks blocks, one after another.  Block j
+ * (numbered params->block + j in the random streams) starts from
+ * dg_init_canvas' noise and runs dg_denoise_loop from k = 0; its committed
+ * canvas is written to blocks[j] before block j + 1 starts.
+ *   blocks       int32 [n_blocks][B*L] device out: the committed blocks.
+ *   steps_taken  HOST int32 [n_blocks][B] out: steps each canvas ran.
+ *   canvas, prev_argmax  int32 [B*L] device scratch (the current block).
+ *   h_buf, accept, entropy, sampled, argmax, stop, workspace: as for
+ *   dg_denoise_loop (the outputs hold the last block's last steps).
+ * Synchronises `stream` once per step (the loop's stop-flag read). */
+dg_status dg_generate_blocks(const dg_shape* shape, const dg_params* params,
+                             const void* E, const float* e_scale, int32_t n_blocks,
+                             dg_block_hidden_fn hidden_fn, void* user, void* h_buf,
+                             int32_t* blocks, int32_t* steps_taken,
+                             int32_t* canvas, int32_t* prev_argmax,
+                             uint8_t* accept, float* entropy, int32_t* sampled,
+                             int32_t* argmax, int32_t* stop,
+                             void* workspace, size_t ws_bytes, void* stream);
+
 /* dg_denoise_step_noalloc -- dg_denoise_step for callers that cannot
  * allocate device memory for a workspace: a serving runtime that has carved
  * up the whole GPU for its own pools, or code that must not call the CUDA
@@ -218,17 +268,20 @@ dg_status dg_denoise_loop(const dg_shape* shape, const dg_params* params,
  * Same arguments and results as dg_denoise_step, without workspace and
  * ws_bytes.  The scratch lives in a fixed 8 MiB array of the library's own
  * device memory, held on every GPU that loads the library until the process
- * exits.  Shapes needing more (dg_workspace_size() > 8 MiB; on a 148-SM B200
- * at d = 2816, V = 262,144 that is B > 4) return DG_ERR_WORKSPACE before
- * anything is launched, with the sizes in dg_last_error_message().  The
- * first call on a device looks the array's device address up once (the
- * runtime may initialise the context then), so make it before any stream
- * capture.  Every call uses the same array: calls that overlap on the GPU
- * (other streams, other threads) race and must be serialised by the caller.
- * Each call clears the parts that must start at zero (fault latch, tickets)
- * on `stream`.  A device-side timeout (or, for the FP8 head, a non-finite
- * h) latches in the array and is cleared by the next call; it is not
- * reported to the caller. */
+ * exits.  Shapes needing more (dg_workspace_size() > 8 MiB) return
+ * DG_ERR_WORKSPACE before anything is launched, with the sizes in
+ * dg_last_error_message(); on a 148-SM B200 at d = 2816, V = 262,144 that
+ * is B > 4 canvases with the bf16 embedder and B > 2 with the FP8 embedder
+ * (whose scratch also holds the two E4M3 terms of h).  All argument checks
+ * run before the array is touched.  The first call on a device looks the
+ * array's device address up once (the runtime may initialise the context
+ * then), so make it before any stream capture.  Every call uses the same
+ * array: calls that overlap on the GPU (other streams, other threads) race
+ * and must be serialised by the caller.  Each call clears, on `stream`, the
+ * parts that must start at zero (tickets, key records).  A device-side
+ * fault (a bounded wait that ran out, or for the FP8 head a non-finite h)
+ * latches in the array and leaves that call's results undefined; the latch
+ * is kept across calls until dg_noalloc_status() reads and clears it. */
 dg_status dg_denoise_step_noalloc(const dg_shape* shape, const dg_params* params,
                                   const void* h, const void* E, const float* e_scale,
                                   const int32_t* step_idx, const uint8_t* has_prev,
@@ -236,6 +289,13 @@ dg_status dg_denoise_step_noalloc(const dg_shape* shape, const dg_params* params
                                   int32_t* canvas, int32_t* prev_argmax,
                                   uint8_t* accept, float* entropy, int32_t* sampled,
                                   int32_t* argmax, int32_t* stop, void* stream);
+
+/* Synchronise `stream`, then read and clear the fault latch of
+ * dg_denoise_step_noalloc's array on the current device: DG_OK (no fault
+ * since the last read), DG_ERR_TIMEOUT, DG_ERR_VALUE or DG_ERR_CUDA, as
+ * dg_device_status() does for a workspace.  Call it after the steps whose
+ * results are to be trusted. */
+dg_status dg_noalloc_status(void* stream);
 
 /* ---- vocabulary-sharded step ---------------------------------------------
  * For an embedder split over G GPUs by vocabulary rows (equal shards of
@@ -297,6 +357,11 @@ dg_status dg_set_head_events(void* ev_start, void* ev_stop);
  * ran out as designed (the context stays usable), DG_OK otherwise. */
 dg_status dg_selftest_bounded_wait(uint64_t limit_ns, void* workspace, size_t ws_bytes,
                                    void* stream);
+
+/* The same self test against the fault latch of dg_denoise_step_noalloc's
+ * array; returns what dg_noalloc_status() then reports (DG_ERR_TIMEOUT when
+ * the wait ran out as designed; the latch is cleared). */
+dg_status dg_noalloc_selftest_bounded_wait(uint64_t limit_ns, void* stream);
 
 /* For n Philox words (device uint32 [n]) write the specified float32
  * Gumbel noise g32 = -L(-L(u)) (device float [n]) and the approximate

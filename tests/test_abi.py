@@ -45,7 +45,7 @@ def test_default_params_are_serving_defaults(libdg):
     assert (p.tau0, p.tau1, p.max_steps, p.entropy_bound, p.stop_entropy) == (0.8, 0.4, 48, 0.1, 0.005)
     # the struct layout of the binding matches the library's (fields after the
     # seed read back as set by the C side)
-    assert (p.seed, p.selection_rule, p.top_k) == (1234, dg.SELECT_CUMSUM, 1)
+    assert (p.seed, p.selection_rule, p.top_k, p.block) == (1234, dg.SELECT_CUMSUM, 1, 0)
 
 
 def test_selection_rule_checks(libdg):
@@ -71,9 +71,9 @@ def test_error_strings(libdg):
     assert libdg.dg_error_string(9) != libdg.dg_error_string(99)
 
 
-def _call_step(libdg, B=1, L=256, d=512, V=8192, ks=(0,), e_dtype=0, null=False, e_scale=None):
+def _call_step(libdg, B=1, L=256, d=512, V=8192, ks=(0,), e_dtype=0, null=False, e_scale=None, params=None):
     shp = dg._Shape(B, L, d, V, e_dtype)
-    prm = dg.Params().c()
+    prm = (params or dg.Params()).c()
     ksa = np.asarray(ks, np.int32)
     hp = np.zeros(max(B, 1), np.uint8)
     fake = ctypes.c_void_p(0 if null else 256)   # never dereferenced: checks fail first
@@ -130,3 +130,30 @@ def test_sharded_entry_points_host_checks(libdg):
     assert libdg.dg_merge_partials(ctypes.byref(shp), ctypes.byref(prm), fake, 2, 0, kp,
                                    hp.ctypes.data_as(ctypes.c_void_p), None, *outs, fake,
                                    ctypes.c_size_t(1 << 30), None) == 1
+
+
+def test_block_index_checks(libdg):
+    # the Philox counter's step word is k | block << 16: a block outside
+    # [0, 65535] or more than 65536 steps are refused on the host
+    assert _call_step(libdg, params=dg.Params(block=65536)) == 1
+    assert _call_step(libdg, params=dg.Params(block=-1)) == 1
+    assert _call_step(libdg, params=dg.Params(max_steps=65537)) == 1
+    shp = dg._Shape(1, 256, 512, 4096, 0)
+    fake = ctypes.c_void_p(256)
+    assert libdg.dg_init_canvas(ctypes.byref(shp), ctypes.byref(dg.Params(block=70000).c()), fake, None) == 1
+    assert libdg.dg_init_canvas(ctypes.byref(shp), ctypes.byref(dg.Params().c()), None, None) == 1
+    bad = dg._Shape(1, 128, 512, 4096, 0)
+    assert libdg.dg_init_canvas(ctypes.byref(bad), ctypes.byref(dg.Params().c()), fake, None) == 2
+    # the generation: at least one block, a callback, outputs; the last
+    # block's index must fit too
+    prm = dg.Params().c()
+    cb = dg._BLOCK_HIDDEN_FN(lambda *a: 0)
+    outs = [fake] * 5
+    args = (fake, fake, fake, fake, *outs, fake, ctypes.c_size_t(1 << 30), None)
+    assert libdg.dg_generate_blocks(ctypes.byref(shp), ctypes.byref(prm), fake, None, 0, cb, None, fake,
+                                    *args) == 1
+    steps = np.zeros(4, np.int32)
+    sp = steps.ctypes.data_as(ctypes.c_void_p)
+    late = dg.Params(block=65534).c()
+    assert libdg.dg_generate_blocks(ctypes.byref(shp), ctypes.byref(late), fake, None, 3, cb, None, fake,
+                                    fake, sp, fake, fake, *outs, fake, ctypes.c_size_t(1 << 30), None) == 1

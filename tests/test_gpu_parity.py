@@ -88,15 +88,35 @@ def test_stop_fires_only_with_previous_prediction():
     compare_with_oracle(g1, h, E, ks, np.ones(1, np.uint8), g0["argmax"], params)
 
 
-def test_inactive_canvas_untouched():
+@pytest.mark.parametrize("B,active", [(2, [1, 0]), (4, [0, 1, 0, 1]), (3, [0, 0, 1])])
+def test_frozen_canvases_untouched_and_active_ones_exact(B, active):
+    # frozen canvases cost no work and keep every output; the updated ones
+    # equal the same canvases of a step that updates every canvas
+    h, E, canvas0 = seeded_inputs(B, 256, 1024)
+    ks = np.array([4 + b for b in range(B)], np.int32)
+    prev = np.full(B * 256, 7, np.int32)
+    hp = np.zeros(B, np.uint8)
+    g = run_step(h, E, ks, hp, prev, canvas0, dg.Params(), active=active, debug=False)
+    full = run_step(h, E, ks, hp, prev, canvas0, dg.Params(), debug=False)
+    for b in range(B):
+        sl = slice(b * 256, (b + 1) * 256)
+        if active[b]:
+            for key in ("canvas", "prev_argmax", "accept", "entropy", "sampled", "argmax"):
+                assert np.array_equal(g[key][sl], full[key][sl]), (b, key)
+            assert g["stop"][b] == full["stop"][b]
+        else:
+            assert np.array_equal(g["canvas"][sl], canvas0[sl])
+            assert np.all(g["prev_argmax"][sl] == 7)
+            assert np.all(g["entropy"][sl] == 0) and np.all(g["sampled"][sl] == 0)
+            assert np.all(g["argmax"][sl] == 0) and np.all(g["accept"][sl] == 0)
+            assert g["stop"][b] == -1
+
+
+def test_every_canvas_frozen_launches_nothing():
     h, E, canvas0 = seeded_inputs(2, 256, 1024)
-    ks = np.array([4, 4], np.int32)
-    prev = np.full(512, 7, np.int32)
-    g = run_step(h, E, ks, np.zeros(2, np.uint8), prev, canvas0, dg.Params(), active=[1, 0])
-    assert np.array_equal(g["canvas"][256:], canvas0[256:])
-    assert np.all(g["prev_argmax"][256:] == 7)
-    assert g["stop"][1] == -1
-    assert not np.array_equal(g["canvas"][:256], canvas0[:256])
+    g = run_step(h, E, [3, 3], np.zeros(2, np.uint8), np.zeros(512, np.int32), canvas0, dg.Params(),
+                 active=[0, 0], debug=False)
+    assert np.array_equal(g["canvas"], canvas0) and np.all(g["stop"] == -1)
 
 
 def test_bounded_wait_selftest_then_step_still_works():

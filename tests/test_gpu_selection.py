@@ -45,11 +45,13 @@ def _low_entropy_case(ks, d=512, V=8192):
     (dg.SELECT_TOPK, 0.1, 256, False),
 ])
 def test_selection_rules_parity_and_replay(rule, bound, k, expect_mid):
-    # steps 3-5: the accepted prefix ends between slot 1 and slot 60, where
-    # the canvases' neighbouring entropies are at least ~1e-6 apart (step 6
-    # puts the cut among entropies ~1e-7 apart, where float32 and float64
-    # entropies order differently and whole swaps exceed the 0.1 % budget)
-    ks = np.array([3, 4, 5], np.int32)
+    # steps 3-6: the accepted prefix ends between slot 1 and slot 60 (steps
+    # 3-5) and near slot 233 (step 6), where the running entropy sum crosses
+    # the bound among slots of entropy ~5e-4 whose cumulative sum is within
+    # 1.4e-5 of the bound: a bias of more than ~6e-8 nats per slot moves the
+    # cut, so this case checks that the entropies of confident slots keep
+    # their full relative precision
+    ks = np.array([3, 4, 5, 6], np.int32)
     h, E, canvas0 = _low_entropy_case(ks)
     B = len(ks)
     hp = np.ones(B, np.uint8)
@@ -63,6 +65,26 @@ def test_selection_rules_parity_and_replay(rule, bound, k, expect_mid):
         assert np.all(counts == k)
     elif expect_mid:
         assert counts.min() >= 1 and np.any((counts > 1) & (counts < L)), counts
+
+
+@pytest.mark.parametrize("rule", [dg.SELECT_CUMSUM, dg.SELECT_MI])
+def test_cut_among_low_entropies_step6(rule):
+    # three canvases at step 6 of the loop stand-in: mean entropy 5.4e-4,
+    # about 233 of 256 slots accepted, the cumulative sum at the cut within
+    # 1.4e-5 to 5.1e-5 of the bound; masks must match the oracle within the
+    # stated budget (at most one slot of the 768)
+    ks = np.array([6, 6, 6], np.int32)
+    h, E, canvas0 = _low_entropy_case(ks)
+    hp = np.ones(3, np.uint8)
+    prev = np.zeros(3 * L, np.int32)
+    params = dg.Params(selection_rule=rule)
+    g = run_step(h, E, ks, hp, prev, canvas0, params)
+    report = {}
+    compare_with_oracle(g, h, E, ks, hp, prev, params, report=report)
+    check_replay(g, ks, hp, prev, params)
+    counts = g["accept"].reshape(3, L).sum(axis=1)
+    assert np.all((counts > 200) & (counts < L)), counts
+    assert report["entropy_max_abs_err"] < 1e-7, report   # confident slots keep their precision
 
 
 def test_mi_rule_accepts_a_superset_of_the_cumsum_rule():

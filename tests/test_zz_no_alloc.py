@@ -16,7 +16,8 @@ import ctypes
 import numpy as np
 import pytest
 
-from dg_testlib import ENTROPY_TOL, seeded_inputs, to_dev_bf16
+import synth
+from dg_testlib import ENTROPY_TOL, seeded_inputs, to_dev_bf16, to_dev_fp8
 
 pytestmark = pytest.mark.gpu
 
@@ -44,49 +45,75 @@ def _args(o):
     return (o["canvas"], o["prev_argmax"], o["accept"], o["entropy"], o["sampled"], o["argmax"], o["stop"])
 
 
-@pytest.mark.parametrize("B,d,V,ks,hp", [
-    (1, 512, 8192, [0], [0]),
-    (2, 2816, 4096, [3, 40], [1, 0]),
-    (1, 2816, 262144, [23], [1]),
+@pytest.mark.parametrize("B,d,V,ks,hp,fp8", [
+    (1, 512, 8192, [0], [0], False),
+    (2, 2816, 4096, [3, 40], [1, 0], False),
+    (1, 2816, 262144, [23], [1], False),
+    (1, 2816, 262144, [23], [1], True),
 ])
-def test_noalloc_matches_workspace_step_on_two_calls(B, d, V, ks, hp):
+def test_noalloc_matches_workspace_step_on_two_calls(B, d, V, ks, hp, fp8):
     h_bits, E_bits, canvas0 = seeded_inputs(B, d, V)
     prev = np.random.default_rng(9).integers(0, V, B * 256).astype(np.int32)
     h = to_dev_bf16(h_bits)
-    E = to_dev_bf16(E_bits)
+    if fp8:
+        E, sc = to_dev_fp8(*synth.quantize_e4m3_rows(E_bits))
+    else:
+        E, sc = to_dev_bf16(E_bits), None
     R = B * 256
     params = dg.Params(seed=4321)
 
-    ws = dg.Workspace(B, d, V)
+    ws = dg.Workspace(B, d, V, dg.E_FP8_E4M3 if fp8 else dg.E_BF16)
     ref = _buffers(R, B, canvas0, prev)
-    dg.denoise_step(h, E, ks, hp, *_args(ref), ws, params)
+    dg.denoise_step(h, E, ks, hp, *_args(ref), ws, params, e_scale=sc)
     torch.cuda.synchronize()
     assert dg.device_status(ws) == 0
     ref = {k: v.cpu().numpy() for k, v in ref.items()}
 
     for call in range(2):
         out = _buffers(R, B, canvas0, prev)
-        dg.denoise_step_noalloc(h, E, ks, hp, *_args(out), params)
+        dg.denoise_step_noalloc(h, E, ks, hp, *_args(out), params, e_scale=sc)
         torch.cuda.synchronize()
+        assert dg.noalloc_status() == 0
         out = {k: v.cpu().numpy() for k, v in out.items()}
         for key in ("canvas", "prev_argmax", "accept", "sampled", "argmax", "stop"):
             assert np.array_equal(out[key], ref[key]), (call, key)
         assert np.abs(out["entropy"].astype(np.float64) - ref["entropy"]).max() <= ENTROPY_TOL, call
 
 
-def test_noalloc_refuses_shapes_beyond_its_scratch():
-    # B = 8 canvases over the 262,144-token vocabulary need about 29 MiB of
-    # scratch: refused up front, so no tensor is touched (the fake pointers
-    # are never dereferenced)
+def _refused(B, e_dtype):
     L = dg.lib()
-    shp = dg._Shape(8, 256, 2816, 262144, 0)
+    shp = dg._Shape(B, 256, 2816, 262144, e_dtype)
     prm = dg.Params().c()
-    ks = np.zeros(8, np.int32)
-    hpv = np.zeros(8, np.uint8)
+    ks = np.zeros(B, np.int32)
+    hpv = np.zeros(B, np.uint8)
     fake = ctypes.c_void_p(256)
-    code = L.dg_denoise_step_noalloc(ctypes.byref(shp), ctypes.byref(prm), fake, fake, None,
+    scale = fake if e_dtype == dg.E_FP8_E4M3 else None
+    return L.dg_denoise_step_noalloc(ctypes.byref(shp), ctypes.byref(prm), fake, fake, scale,
                                      ks.ctypes.data_as(ctypes.c_void_p), hpv.ctypes.data_as(ctypes.c_void_p),
                                      None, fake, fake, fake, fake, fake, fake, fake, None)
+
+
+@pytest.mark.parametrize("B,e_dtype", [(8, dg.E_BF16), (5, dg.E_BF16), (3, dg.E_FP8_E4M3)])
+def test_noalloc_refuses_shapes_beyond_its_scratch(B, e_dtype):
+    # over the 262,144-token vocabulary, B = 5 bf16 canvases need about
+    # 8.8 MiB of scratch (B = 8: about 14 MiB) and B = 3 with the FP8
+    # embedder about 9.4 MiB (its scratch also holds h's two E4M3 terms):
+    # refused before anything runs, so the fake pointers are never touched
+    code = _refused(B, e_dtype)
     assert code == 3    # DG_ERR_WORKSPACE
-    msg = L.dg_last_error_message().decode()
+    msg = dg.lib().dg_last_error_message().decode()
     assert "scratch" in msg and "bytes" in msg
+
+
+def test_noalloc_reports_a_latched_fault_then_runs_clean():
+    # the bounded-wait self test latches a timeout in the shared array (it
+    # gives up after 2 ms, nothing hangs); the status call reports it once
+    # and clears it, and the next step runs with a clean latch
+    assert dg.noalloc_selftest_bounded_wait(2_000_000) == 6   # DG_ERR_TIMEOUT
+    assert dg.noalloc_status() == 0
+    B, d, V = 1, 512, 8192
+    h_bits, E_bits, canvas0 = seeded_inputs(B, d, V)
+    out = _buffers(256, B, canvas0, np.zeros(256, np.int32))
+    dg.denoise_step_noalloc(to_dev_bf16(h_bits), to_dev_bf16(E_bits), [0], [0], *_args(out))
+    assert dg.noalloc_status() == 0
+    assert int(out["accept"].sum()) >= 1
