@@ -20,7 +20,8 @@ its own step index drawn uniformly from [0, 47] (seed 5) and advanced by one
 every step; at B >= 8 the step is bound by the tensor cores and the roofline
 object says so.  The default B = 1 line also reports the adaptive loop run
 once, untimed, at the production shape on the synthetic stand-in hidden
-states (the step at which it stops).
+states (the step at which it stops); so does every --batch / --e-dtype
+line, for its B canvases.
 
 For N > 1 launch with torch.distributed.run; each rank runs its own canvas
 (replicas, no data-path collective): weak scaling.  ``--impl reference``
@@ -262,42 +263,48 @@ def run_reference(args):
     return 0
 
 
-def loop_report(dg, E, E_bits, e_scale, fp8, ws_dtype, torch):
-    """The adaptive loop once at the production shape (B = 1), untimed: the
-    synthetic stand-in hidden states of the loop configuration (signal
-    growing with k, targets seed 3, noise seed 4 + k), generated on the host
-    each step and copied in.  Returns the step count at stop with the
-    per-step mean entropy and accepted slots."""
+def loop_report(dg, E, E_bits, e_scale, fp8, ws_dtype, torch, B=1):
+    """The adaptive loop once at the production shape, untimed, for B
+    canvases: the synthetic stand-in hidden states of the loop configuration
+    (signal growing with k, targets seed 3, noise seed 4 + k), generated on
+    the host each step and copied in.  Returns the steps each canvas ran
+    until it stopped, with the per-step mean entropy and accepted slots."""
     import synth
-    y = synth.loop_targets(L, V, seed=3)
-    h_buf = torch.empty((L, D), dtype=torch.bfloat16, device="cuda")
-    canvas = torch.from_numpy(synth.canvas_uniform(1, L, V, seed=0)).cuda()
-    prev = torch.zeros(L, dtype=torch.int32, device="cuda")
-    hp = np.zeros(1, np.uint8)
-    acc = torch.zeros(L, dtype=torch.uint8, device="cuda")
-    ent = torch.zeros(L, dtype=torch.float32, device="cuda")
-    samp = torch.zeros(L, dtype=torch.int32, device="cuda")
-    amax = torch.zeros(L, dtype=torch.int32, device="cuda")
-    stop = torch.zeros(1, dtype=torch.int32, device="cuda")
-    ws = dg.Workspace(1, D, V, ws_dtype)
+    R = B * L
+    y = synth.loop_targets(L, V, seed=3, B=B)
+    h_buf = torch.empty((R, D), dtype=torch.bfloat16, device="cuda")
+    canvas = torch.from_numpy(synth.canvas_uniform(B, L, V, seed=0)).cuda()
+    prev = torch.zeros(R, dtype=torch.int32, device="cuda")
+    hp = np.zeros(B, np.uint8)
+    acc = torch.zeros(R, dtype=torch.uint8, device="cuda")
+    ent = torch.zeros(R, dtype=torch.float32, device="cuda")
+    samp = torch.zeros(R, dtype=torch.int32, device="cuda")
+    amax = torch.zeros(R, dtype=torch.int32, device="cuda")
+    stop = torch.zeros(B, dtype=torch.int32, device="cuda")
+    ws = dg.Workspace(B, D, V, ws_dtype)
     trace = []
+
+    def note():
+        trace[-1]["mean_entropy"] = float(ent.mean())
+        trace[-1]["accepted"] = int(acc.sum())
 
     def hidden(k, canvas_t, h_t):
         if trace:   # the previous step's results are final once this runs
-            trace[-1]["mean_entropy"] = float(ent.mean())
-            trace[-1]["accepted"] = int(acc.sum())
+            note()
         h_t.copy_(torch.from_numpy(synth.loop_hidden(k, y, E_bits, seed=4).view(np.int16)).view(torch.bfloat16))
         trace.append({"k": int(k)})
 
     steps = dg.denoise_loop(E, hidden, h_buf, canvas, prev, hp, acc, ent, samp, amax, stop, ws,
                             dg.Params(), e_scale=e_scale)
     torch.cuda.synchronize()
-    trace[-1]["mean_entropy"] = float(ent.mean())
-    trace[-1]["accepted"] = int(acc.sum())
+    note()
     match = float((canvas.cpu().numpy() == y).mean())
-    return {"steps_at_stop": int(steps[0]), "stopped_early": bool(int(steps[0]) < 48),
-            "per_step": trace, "committed_equals_targets": match,
-            "workload": "B=1, L=256, d=2816, V=262144, stand-in h_i = (k/12) 3 E[y_i]/|E[y_i]| sqrt(d) + N(0,1)"}
+    return {"steps_at_stop": int(steps.max()) if B == 1 else [int(v) for v in np.bincount(steps)],
+            "steps_at_stop_is": "steps run" if B == 1 else "histogram over canvases of the steps each ran",
+            "stopped_early": bool(int(steps.max()) < 48), "per_step": trace,
+            "committed_equals_targets": match,
+            "workload": f"B={B}, L=256, d=2816, V=262144, {'E4M3' if fp8 else 'bf16'} embedder, stand-in "
+                        "h_i = (k/12) 3 E[y_i]/|E[y_i]| sqrt(d) + N(0,1)"}
 
 
 def main():
@@ -455,8 +462,8 @@ def main():
     e2e_value = world * B * L / (e2e_ms / 1e3)
 
     loop = None
-    if B == 1 and world == 1 and not args.no_loop:
-        loop = loop_report(dg, E, E_bits, e_scale, fp8, ws_dtype, torch)
+    if world == 1 and not args.no_loop:
+        loop = loop_report(dg, E, E_bits, e_scale, fp8, ws_dtype, torch, B)
 
     if rank == 0:
         pk, pk_kind = peaks()

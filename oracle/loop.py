@@ -19,19 +19,23 @@ from .step import Params, denoise_step
 
 def denoise_loop(hidden_fn, *, E_bits=None, q=None, s=None, B: int, L: int = 256,
                  params: Params = Params(), k_start: int = 0, canvas=None,
-                 prev_argmax=None, has_prev=None):
+                 prev_argmax=None, has_prev=None, canvases=None):
     """Run steps k_start .. N-1 until every canvas stops.
 
     ``hidden_fn(k, canvas)`` returns the bf16 hidden-state bits [B*L, d] of
     step k.  Returns (final canvas int32 [B*L], steps taken int32 [B], the
-    per-step history of stop flags and mean entropies).
+    per-step history of stop flags and mean entropies).  With ``canvases``
+    only those canvases of the batch are run (canvases are independent: each
+    has its own random streams); the others keep their input canvas and 0
+    steps.
     """
     N = params.max_steps
     V = (E_bits if E_bits is not None else q).shape[0]
     canvas = np.zeros(B * L, np.int32) if canvas is None else np.array(canvas, np.int32)
     prev = np.zeros(B * L, np.int32) if prev_argmax is None else np.array(prev_argmax, np.int32)
     hp = np.zeros(B, np.uint8) if has_prev is None else np.array(has_prev, np.uint8)
-    active = np.ones(B, dtype=bool)
+    active = np.zeros(B, dtype=bool)
+    active[list(range(B)) if canvases is None else [int(c) for c in canvases]] = True
     steps = np.zeros(B, np.int32)
     history = []
     for k in range(k_start, N):

@@ -135,3 +135,15 @@ def test_freeze_check_rejects_a_loop_that_keeps_updating_a_stopped_canvas():
     bad_fin[256 + 3] = (bad_fin[256 + 3] + 1) % 1024
     with pytest.raises(AssertionError):
         check_freeze_and_commit(E, bad_fin, steps, seen, hs, p)
+
+
+def test_loop_over_a_subset_of_canvases_equals_the_full_loop_on_them():
+    E = synth.embedder_normal(1024, 256, seed=1)
+    y = synth.loop_targets(256, 1024, seed=3, B=3)
+    hidden = lambda k, c: synth.loop_hidden(k, y, E, seed=4)   # noqa: E731
+    full, steps, _ = denoise_loop(hidden, E_bits=E, B=3, L=256)
+    sub, ssteps, _ = denoise_loop(hidden, E_bits=E, B=3, L=256, canvases=[2, 0])
+    for b in (0, 2):
+        assert np.array_equal(sub[b * 256:(b + 1) * 256], full[b * 256:(b + 1) * 256])
+        assert ssteps[b] == steps[b]
+    assert ssteps[1] == 0 and np.all(sub[256:512] == 0)
