@@ -19,7 +19,8 @@ __all__ = ["DGError", "Params", "lib", "workspace_size", "Workspace", "denoise_s
            "selftest_bounded_wait", "set_head_events", "denoise_step_noalloc", "noalloc_status",
            "noalloc_selftest_bounded_wait", "STATUS", "E_BF16", "E_FP8_E4M3",
            "SELECT_CUMSUM", "SELECT_MI", "SELECT_TOPK", "partials_count", "head_partials", "merge_partials",
-           "gather_partials", "init_canvas", "generate_blocks"]
+           "gather_partials", "init_canvas", "generate_blocks", "loop_state_bytes", "LoopState",
+           "denoise_loop_graph"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdg.so")
@@ -115,6 +116,12 @@ def lib() -> ctypes.CDLL:
         L.dg_noalloc_selftest_bounded_wait.argtypes = [ctypes.c_uint64, P]
         L.dg_noalloc_selftest_bounded_wait.restype = ctypes.c_int
         L.dg_last_error_message.restype = ctypes.c_char_p
+        L.dg_loop_state_bytes.argtypes = [ctypes.c_int32]
+        L.dg_loop_state_bytes.restype = ctypes.c_size_t
+        L.dg_denoise_loop_graph.argtypes = [ctypes.POINTER(_Shape), ctypes.POINTER(_Params), P, P, P,
+                                            ctypes.c_int32, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P,
+                                            ctypes.c_size_t, P]
+        L.dg_denoise_loop_graph.restype = ctypes.c_int
         L.dg_init_canvas.argtypes = [ctypes.POINTER(_Shape), ctypes.POINTER(_Params), P, P]
         L.dg_init_canvas.restype = ctypes.c_int
         L.dg_generate_blocks.argtypes = [ctypes.POINTER(_Shape), ctypes.POINTER(_Params), P, P, ctypes.c_int32,
@@ -304,6 +311,54 @@ def denoise_loop(E, hidden_fn, h_buf, canvas, prev_argmax, has_prev, accept, ent
         if errors:
             raise err from errors[0]
         raise err
+    return steps
+
+
+def loop_state_bytes(B: int) -> int:
+    """Bytes of device loop state ``dg_denoise_loop_graph`` needs for B canvases."""
+    return int(lib().dg_loop_state_bytes(ctypes.c_int32(B)))
+
+
+class LoopState:
+    """Device loop state of the device-side loop (a torch uint8 buffer);
+    ``k`` is a one-element int32 view of the step index the loop's graph
+    body is about to run, for a hidden-state graph to read."""
+
+    def __init__(self, B: int, device=None):
+        import torch
+        n = loop_state_bytes(B)
+        if n == 0:
+            raise DGError(1, "loop_state_bytes")
+        self.nbytes = n
+        self.buf = torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+        self.k = self.buf[:4].view(torch.int32)
+
+
+def denoise_loop_graph(E, hidden_graph, h_buf, canvas, prev_argmax, has_prev, accept, entropy, sampled,
+                       argmax, stop, ws: Workspace, state: LoopState, params: Params = Params(),
+                       k_start: int = 0, e_scale=None, stream=None):
+    """The adaptive loop run on the device (``dg_denoise_loop_graph``).
+
+    ``hidden_graph`` is a ``torch.cuda.CUDAGraph`` captured with
+    ``keep_graph=True`` that writes step ``state.k``'s hidden states into
+    ``h_buf`` (or None: ``h_buf`` stays as it is).  ``has_prev`` is a host
+    uint8 numpy array [B] updated in place.  Returns the host int32 array of
+    steps taken."""
+    B = int(len(has_prev))
+    R, d = h_buf.shape
+    V = E.shape[0]
+    e_dtype = E_BF16 if e_scale is None else E_FP8_E4M3
+    shp = _shape(B, d, V, e_dtype, L=R // B)
+    prm = params.c()
+    steps = np.zeros(B, np.int32)
+    assert isinstance(has_prev, np.ndarray) and has_prev.dtype == np.uint8
+    g = None if hidden_graph is None else ctypes.c_void_p(int(hidden_graph.raw_cuda_graph()))
+    _check(lib().dg_denoise_loop_graph(
+        ctypes.byref(shp), ctypes.byref(prm), _ptr(E), _ptr(e_scale), g, ctypes.c_int32(k_start), _ptr(h_buf),
+        _ptr(canvas), _ptr(prev_argmax), has_prev.ctypes.data_as(ctypes.c_void_p),
+        steps.ctypes.data_as(ctypes.c_void_p), _ptr(accept), _ptr(entropy), _ptr(sampled), _ptr(argmax),
+        _ptr(stop), _ptr(state.buf), ctypes.c_size_t(state.nbytes), _ptr(ws.buf), ctypes.c_size_t(ws.nbytes),
+        _stream(stream)), "dg_denoise_loop_graph")
     return steps
 
 

@@ -136,6 +136,7 @@ struct StepArgs {
   float* part_out = nullptr;      // head only: the records [7][R][P] go here
   const float* part_in = nullptr; // merge only: S shards' records [S][7][R][P]
   int32_t S = 1, P = 0;           // merge only
+  const LoopDevState* loop = nullptr;  // device-side loop: per-canvas data from device memory
 };
 
 // Every check of a step's arguments except those of the workspace: shape,
@@ -273,11 +274,15 @@ dg_status run_step(const StepArgs& a) {
     hp.wait_ns = kDefaultWaitNs;
     memcpy(hp.cp, cps, sizeof(cps));
 
-    if (t_head_ev_start != nullptr && cudaEventRecord(t_head_ev_start, a.stream) != cudaSuccess)
-      return DG_ERR_CUDA;
+    if (a.loop != nullptr) {
+      hp.cp_dev = a.loop->cp;
+      hp.mtile_dev = a.loop->canvas_of;
+      hp.mt_dev = a.loop->n_active;
+    }
+    const bool events = t_head_ev_start != nullptr && a.loop == nullptr;
+    if (events && cudaEventRecord(t_head_ev_start, a.stream) != cudaSuccess) return DG_ERR_CUDA;
     if (!cuda_ok(launch_head(fp8, tmA, tmA2, tmB, hp, a.stream), "head kernel launch")) return DG_ERR_CUDA;
-    if (t_head_ev_stop != nullptr && cudaEventRecord(t_head_ev_stop, a.stream) != cudaSuccess)
-      return DG_ERR_CUDA;
+    if (events && cudaEventRecord(t_head_ev_stop, a.stream) != cudaSuccess) return DG_ERR_CUDA;
   }
   if (!merge) return DG_OK;
 
@@ -306,11 +311,32 @@ dg_status run_step(const StepArgs& a) {
   mp.stop_entropy = pr.stop_entropy;
   memcpy(mp.cp, cps, sizeof(cps));
   memcpy(mp.canvas_of, upd, sizeof(upd));
-  if (!cuda_ok(launch_merge(mp, a.stream), "merge kernel launch")) return DG_ERR_CUDA;
+  if (a.loop != nullptr) {
+    mp.cp_dev = a.loop->cp;
+    mp.canvas_of_dev = a.loop->canvas_of;
+    mp.n_dev = a.loop->n_active;
+  }
+  if (!cuda_ok(launch_merge(mp, a.stream, a.loop == nullptr), "merge kernel launch")) return DG_ERR_CUDA;
   return DG_OK;
 }
 
 }  // namespace
+
+dg_status enqueue_loop_step(const dg_shape* shape, const dg_params* params, const void* h, const void* E,
+                            const float* e_scale, int32_t k_any, int32_t* canvas, int32_t* prev_argmax,
+                            uint8_t* accept, float* entropy, int32_t* sampled, int32_t* argmax, int32_t* stop,
+                            void* workspace, size_t ws_bytes, const LoopDevState* loop, cudaStream_t stream) {
+  int32_t ks[DG_MAX_B];
+  uint8_t hp[DG_MAX_B];
+  for (int b = 0; b < DG_MAX_B; ++b) {
+    ks[b] = k_any;
+    hp[b] = 0;
+  }
+  StepArgs a{shape,  params,  h,       E,      e_scale, ks,      hp,        nullptr,  canvas, prev_argmax,
+             accept, entropy, sampled, argmax, stop,    nullptr, workspace, ws_bytes, stream};
+  a.loop = loop;
+  return run_step(a);
+}
 
 dg_status check_shape_and_params(const dg_shape* shape, const dg_params* params) {
   const dg_status st = check_shape(shape);

@@ -91,6 +91,12 @@ struct HeadParams {
   uint32_t rk0[10], rk1[10];  // Philox round keys of the seed
   CanvasParam cp[DG_MAX_B];
   uint8_t mtile[DG_MAX_B];     // canvas of row tile m (m < split.MT)
+  // Device-side loop: when set, the per-canvas data, the row tiles' canvases
+  // and their number are read from device memory (written by the loop's
+  // control kernel) instead of cp, mtile and split.MT.
+  const CanvasParam* cp_dev;
+  const uint8_t* mtile_dev;
+  const int32_t* mt_dev;
 };
 
 struct MergeParams {
@@ -115,6 +121,11 @@ struct MergeParams {
   int32_t top_k;
   CanvasParam cp[DG_MAX_B];
   uint8_t canvas_of[DG_MAX_B];  // canvas of block group g (32 CTAs per canvas)
+  // Device-side loop: per-canvas data, the canvases to update and their
+  // number from device memory; block groups past the number exit at once.
+  const CanvasParam* cp_dev;
+  const uint8_t* canvas_of_dev;
+  const int32_t* n_dev;
 };
 
 // kblock: K elements per stage (kBlockK, or kBlockKFp8 for the FP8 head);
@@ -122,6 +133,23 @@ struct MergeParams {
 // q_cap units per row tile (the records per row the workspace holds).
 HeadSplit head_split(int R, int V, int d, int max_pairs, int kblock, int q_cap = 1 << 30);
 int head_max_pairs(bool fp8);
+
+// Device memory of the device-side loop (inside the caller's loop-state
+// buffer): the per-canvas data of the step about to run, the canvases still
+// running (canvas_of[0 .. *n_active - 1]) and their number.
+struct LoopDevState {
+  CanvasParam* cp;
+  uint8_t* canvas_of;
+  int32_t* n_active;
+};
+
+// Enqueue one step whose per-canvas data come from `loop` (device memory)
+// with every canvas's work split prepared, as the device-side loop's graph
+// body does; k_any is any valid step index (used for the host-side checks).
+dg_status enqueue_loop_step(const dg_shape* shape, const dg_params* params, const void* h, const void* E,
+                            const float* e_scale, int32_t k_any, int32_t* canvas, int32_t* prev_argmax,
+                            uint8_t* accept, float* entropy, int32_t* sampled, int32_t* argmax, int32_t* stop,
+                            void* workspace, size_t ws_bytes, const LoopDevState* loop, cudaStream_t stream);
 
 // Workspace layout (byte offsets), see dg_workspace_size().
 struct WsLayout {
@@ -158,7 +186,9 @@ cudaError_t launch_head(bool fp8, const CUtensorMap& tmA, const CUtensorMap& tmA
 // kErrHiddenRange in *err if some h is not finite.
 cudaError_t launch_hidden_split(const void* h, uint8_t* h1, uint8_t* h2, float* rinv, int R, int d,
                                 uint32_t* err, cudaStream_t stream);
-cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream);
+// pdl: launch as a programmatic dependent of the preceding kernel (the
+// head); off inside graphs built by the device-side loop.
+cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream, bool pdl = true);
 // canvas[b * L + s] = (r V) >> 32, r = Philox word 0 of counter
 // (0, s | 3 << 16, ctr_step, b): the uniform noise a block starts from.
 cudaError_t launch_init_canvas(int32_t* canvas, int B, int L, int V, uint32_t ctr_step, uint32_t seed_lo,

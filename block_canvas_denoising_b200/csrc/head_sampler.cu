@@ -49,12 +49,23 @@ namespace dg {
 
 namespace {
 
+// Row tiles this launch covers, and the per-canvas data: from device memory
+// in the device-side loop, else from the launch parameters.
+DG_DEV int row_tiles(const HeadParams& p) { return p.mt_dev != nullptr ? __ldcg(p.mt_dev) : p.split.MT; }
+DG_DEV CanvasParam canvas_param(const HeadParams& p, int b) {
+  if (p.cp_dev == nullptr) return p.cp[b];
+  CanvasParam c;
+  c.k = __ldcg(&p.cp_dev[b].k);
+  c.inv_tau = __ldcg(&p.cp_dev[b].inv_tau);
+  return c;
+}
+
 // Unit u: row tile (canvas) m, vocabulary tiles [n0, n1), unit index q
-// within the row tile.
-DG_DEV void unit_range(const HeadParams& p, int u, int& m, int& n0, int& n1, int& q) {
+// within the row tile; mt = row_tiles(p).
+DG_DEV void unit_range(const HeadParams& p, int mt, int u, int& m, int& n0, int& n1, int& q) {
   const HeadSplit& sp = p.split;
-  q = u / sp.MT;
-  m = p.mtile[u - q * sp.MT];
+  q = u / mt;
+  m = p.mtile_dev != nullptr ? static_cast<int>(__ldcg(p.mtile_dev + (u - q * mt))) : p.mtile[u - q * mt];
   n0 = static_cast<int>((static_cast<int64_t>(q) * sp.NT) / sp.Q);
   n1 = static_cast<int>((static_cast<int64_t>(q + 1) * sp.NT) / sp.Q);
 }
@@ -312,6 +323,8 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   const int pair = blockIdx.x >> 1;
   const int npairs = gridDim.x >> 1;
   const HeadSplit& sp = p.split;
+  const int mt = row_tiles(p);       // row tiles (canvases) of this launch
+  const int units = mt * sp.Q;
 
   auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
   auto empty_bar = [&](int s) { return smem_u32(&bars[kStages + s]); };
@@ -358,9 +371,9 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int u = pair; u < sp.units && ok; u += npairs) {
+      for (int u = pair; u < units && ok; u += npairs) {
         int m, n0, n1, q;
-        unit_range(p, u, m, n0, n1, q);
+        unit_range(p, mt, u, m, n0, n1, q);
         for (int n = n0; n < n1 && ok; ++n) {
           for (int kb = 0; kb < sp.KB; ++kb) {
             if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, p.wait_ns)) {
@@ -417,9 +430,9 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       uint32_t phase = 0;
       int tile = 0;
       bool ok = true;
-      for (int u = pair; u < sp.units && ok; u += npairs) {
+      for (int u = pair; u < units && ok; u += npairs) {
         int m, n0, n1, q;
-        unit_range(p, u, m, n0, n1, q);
+        unit_range(p, mt, u, m, n0, n1, q);
         for (int n = n0; n < n1 && ok; ++n, ++tile) {
           const int acc = tile & 1;
           const uint32_t acc_phase = (tile >> 1) & 1;
@@ -495,7 +508,8 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         const int hb = hrow >> 8;
         uint32_t w[8];
         const PhiloxRow pr = philox_row(static_cast<uint32_t>(hrow & 255) | (kPurposeGumbel << 16),
-                                        static_cast<uint32_t>(p.cp[hb].k), static_cast<uint32_t>(hb), p.rk0, p.rk1);
+                                        static_cast<uint32_t>(canvas_param(p, hb).k), static_cast<uint32_t>(hb), p.rk0,
+                                        p.rk1);
         philox_words8(static_cast<uint32_t>(p.v_off + n_t * kBlockN + g * 8) >> 2, pr, p.rk0, p.rk1, w);
         dst[g * 32 + r] = max(max(max(w[0], w[1]), max(w[2], w[3])), max(max(w[4], w[5]), max(w[6], w[7])));
       }
@@ -507,18 +521,18 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     // a failed wait (it then skips the work), so the barriers cannot deadlock.
     int tile = 0;
     bool ok = true;
-    if (!mma_quarter) {
+    if (!mma_quarter && pair < units) {
       int m, n0, n1, q;
-      unit_range(p, pair, m, n0, n1, q);
+      unit_range(p, mt, pair, m, n0, n1, q);
       ok = produce_words(0, m, n0);
     }
-    for (int u = pair; u < sp.units; u += npairs) {
+    for (int u = pair; u < units; u += npairs) {
       int m, n0, n1, q;
-      unit_range(p, u, m, n0, n1, q);
+      unit_range(p, mt, u, m, n0, n1, q);
       const int row = m * kPairM + static_cast<int>(rank) * kBlockM + rloc;
       const int b = row >> 8;
       const int slot = row & 255;
-      const CanvasParam cp = p.cp[b];
+      const CanvasParam cp = canvas_param(p, b);
       const float inv_tau = cp.inv_tau;
       const float rinv = kFp8 ? __ldg(p.row_inv + row) : 1.0f;
       const float c2 = __fmul_rn(inv_tau, kLog2e);
@@ -540,9 +554,9 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           // the words of the next tile (this unit's next, or the next unit's first)
           int mn = m, nn = n + 1;
           bool more = nn < n1;
-          if (!more && u + npairs < sp.units) {
+          if (!more && u + npairs < units) {
             int n1n, qn;
-            unit_range(p, u + npairs, mn, nn, n1n, qn);
+            unit_range(p, mt, u + npairs, mn, nn, n1n, qn);
             more = true;
           }
           if (more && !produce_words(tile + 1, mn, nn)) {

@@ -66,7 +66,16 @@ merge_select_kernel(const __grid_constant__ MergeParams p) {
   const int warp = t >> 5;
   const int lane = t & 31;
   constexpr int kCtasPerCanvas = 256 / kRowsPerCta;
-  const int b = p.canvas_of[blockIdx.x / kCtasPerCanvas];  // only the canvases this step updates
+  const int grp = blockIdx.x / kCtasPerCanvas;
+  int b;  // only the canvases this step updates
+  if (p.canvas_of_dev != nullptr) {
+    // device-side loop: the launch covers every canvas; the loop's control
+    // kernel lists the ones still running
+    if (grp >= __ldcg(p.n_dev)) return;
+    b = __ldcg(p.canvas_of_dev + grp);
+  } else {
+    b = p.canvas_of[grp];
+  }
   const int row = b * 256 + (blockIdx.x % kCtasPerCanvas) * kRowsPerCta + warp;
   const size_t plane = static_cast<size_t>(p.R) * p.P;
 
@@ -112,7 +121,13 @@ merge_select_kernel(const __grid_constant__ MergeParams p) {
   if (!s_last) return;
   __threadfence();
 
-  const CanvasParam cp = p.cp[b];
+  CanvasParam cp;
+  if (p.cp_dev != nullptr) {
+    cp.k = __ldcg(&p.cp_dev[b].k);
+    cp.has_prev = __ldcg(&p.cp_dev[b].has_prev);
+  } else {
+    cp = p.cp[b];
+  }
   const int s = t;  // slot
   const int grow = b * 256 + s;
   const float H = __ldcg(p.entropy + grow);
@@ -178,7 +193,7 @@ merge_select_kernel(const __grid_constant__ MergeParams p) {
   if (t == 0) p.stop[b] = stop ? 1 : 0;
 }
 
-cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream) {
+cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream, bool pdl) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.B * (256 / kRowsPerCta), 1, 1);  // p.B: canvases updated
   cfg.blockDim = dim3(256, 1, 1);
@@ -190,7 +205,7 @@ cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream) {
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, merge_select_kernel, p);
 }
 

@@ -219,6 +219,43 @@ dg_status dg_denoise_loop(const dg_shape* shape, const dg_params* params,
                           int32_t* argmax, int32_t* stop,
                           void* workspace, size_t ws_bytes, void* stream);
 
+/* ---- the adaptive loop on the device -------------------------------------
+ * dg_denoise_loop reads the stop flags back to the host after every step.
+ * dg_denoise_loop_graph runs the same loop as one CUDA graph: a conditional
+ * (while) node whose body is [hidden_graph] -> step -> loop control, where a
+ * control kernel commits and freezes the canvases that stopped (or reached
+ * k = max_steps-1), advances k, prepares the next step's temperatures and
+ * the list of canvases still running, and ends the loop when none is left;
+ * nothing returns to the host until the loop is over.  Results equal
+ * dg_denoise_loop's for the same hidden states. */
+
+/* Bytes of device loop state for B canvases (256-byte aligned buffer,
+ * owned by the caller); 0 for B outside [1, DG_MAX_B].  Its first int32 is
+ * the step index k the graph body is about to run: the hidden-state graph
+ * reads it there to produce step k's hidden states. */
+size_t dg_loop_state_bytes(int32_t B);
+
+/* hidden_graph  a cudaGraph_t (or NULL) embedded at the head of the loop
+ *               body: it must write the bf16 [B*L, d] hidden states of step
+ *               k (k = the first int32 of loop_state) into h_buf, using only
+ *               node kinds a conditional body accepts (kernels, memcpy,
+ *               memset).  NULL: h_buf is used as it stands every step.
+ * has_prev      HOST uint8 [B] in/out, as for dg_denoise_loop.
+ * steps_taken   HOST int32 [B] out.
+ * loop_state    device buffer of dg_loop_state_bytes(B) bytes.
+ * Other arguments as for dg_denoise_loop.  The graph is built, run and
+ * destroyed inside the call, which returns after synchronising `stream`; a
+ * device-side fault ends the loop and is returned (DG_ERR_TIMEOUT or
+ * DG_ERR_VALUE). */
+dg_status dg_denoise_loop_graph(const dg_shape* shape, const dg_params* params,
+                                const void* E, const float* e_scale, void* hidden_graph,
+                                int32_t k_start, void* h_buf, int32_t* canvas, int32_t* prev_argmax,
+                                uint8_t* has_prev, int32_t* steps_taken,
+                                uint8_t* accept, float* entropy, int32_t* sampled,
+                                int32_t* argmax, int32_t* stop,
+                                void* loop_state, size_t state_bytes,
+                                void* workspace, size_t ws_bytes, void* stream);
+
 /* ---- block-by-block generation ([Report] Figure 4: encode & append) ----
  * Generation runs block after block: each block of B canvases starts from
  * uniform noise, the adaptive loop denoises it until it settles, and the

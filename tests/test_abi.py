@@ -157,3 +157,28 @@ def test_block_index_checks(libdg):
     late = dg.Params(block=65534).c()
     assert libdg.dg_generate_blocks(ctypes.byref(shp), ctypes.byref(late), fake, None, 3, cb, None, fake,
                                     fake, sp, fake, fake, *outs, fake, ctypes.c_size_t(1 << 30), None) == 1
+
+
+def test_device_loop_host_checks(libdg):
+    # state size, alignment, step range and null arguments are refused on
+    # the host before any device work
+    assert libdg.dg_loop_state_bytes(0) == 0 and libdg.dg_loop_state_bytes(257) == 0
+    n1 = libdg.dg_loop_state_bytes(1)
+    assert n1 >= 256 + 12 and n1 % 256 == 0
+    shp = dg._Shape(1, 256, 512, 4096, 0)
+    fake = ctypes.c_void_p(4096)
+    hp = np.zeros(1, np.uint8)
+    st = np.zeros(1, np.int32)
+    hpp, stp = hp.ctypes.data_as(ctypes.c_void_p), st.ctypes.data_as(ctypes.c_void_p)
+
+    def call(k_start=0, state=fake, nbytes=n1, hpv=hpp, prm=dg.Params()):
+        p = prm.c()
+        return libdg.dg_denoise_loop_graph(ctypes.byref(shp), ctypes.byref(p), fake, None, None, k_start, fake,
+                                           fake, fake, hpv, stp, fake, fake, fake, fake, fake, state,
+                                           ctypes.c_size_t(nbytes), fake, ctypes.c_size_t(1 << 30), None)
+    assert call(k_start=48) == 4
+    assert call(k_start=-1) == 4
+    assert call(state=ctypes.c_void_p(4096 + 16)) == 1     # not 256-byte aligned
+    assert call(nbytes=n1 - 1) == 3
+    assert call(hpv=None) == 1
+    assert call(prm=dg.Params(max_steps=0)) == 1
