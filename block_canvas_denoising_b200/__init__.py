@@ -20,7 +20,7 @@ __all__ = ["DGError", "Params", "lib", "workspace_size", "Workspace", "denoise_s
            "noalloc_selftest_bounded_wait", "STATUS", "E_BF16", "E_FP8_E4M3",
            "SELECT_CUMSUM", "SELECT_MI", "SELECT_TOPK", "partials_count", "head_partials", "merge_partials",
            "gather_partials", "init_canvas", "generate_blocks", "loop_state_bytes", "LoopState",
-           "denoise_loop_graph"]
+           "denoise_loop_graph", "selfcond_workspace_size", "embedder_transpose", "denoise_step_selfcond"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdg.so")
@@ -116,6 +116,13 @@ def lib() -> ctypes.CDLL:
         L.dg_noalloc_selftest_bounded_wait.argtypes = [ctypes.c_uint64, P]
         L.dg_noalloc_selftest_bounded_wait.restype = ctypes.c_int
         L.dg_last_error_message.restype = ctypes.c_char_p
+        L.dg_selfcond_workspace_size.argtypes = [ctypes.POINTER(_Shape)]
+        L.dg_selfcond_workspace_size.restype = ctypes.c_size_t
+        L.dg_embedder_transpose.argtypes = [ctypes.POINTER(_Shape), P, P, P]
+        L.dg_embedder_transpose.restype = ctypes.c_int
+        L.dg_denoise_step_selfcond.argtypes = [ctypes.POINTER(_Shape), ctypes.POINTER(_Params), P, P, P, P, P, P,
+                                               P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+        L.dg_denoise_step_selfcond.restype = ctypes.c_int
         L.dg_loop_state_bytes.argtypes = [ctypes.c_int32]
         L.dg_loop_state_bytes.restype = ctypes.c_size_t
         L.dg_denoise_loop_graph.argtypes = [ctypes.POINTER(_Shape), ctypes.POINTER(_Params), P, P, P,
@@ -172,12 +179,19 @@ def workspace_size(B: int, d: int, V: int, e_dtype: int = E_BF16, L: int = 256) 
     return int(lib().dg_workspace_size(ctypes.byref(_shape(B, d, V, e_dtype, L))))
 
 
-class Workspace:
-    """Device scratch for steps of one shape (a zeroed torch uint8 buffer)."""
+def selfcond_workspace_size(B: int, d: int, V: int, e_dtype: int = E_BF16, L: int = 256) -> int:
+    """Bytes of workspace a step with the self-conditioning signal needs."""
+    return int(lib().dg_selfcond_workspace_size(ctypes.byref(_shape(B, d, V, e_dtype, L))))
 
-    def __init__(self, B: int, d: int, V: int, e_dtype: int = E_BF16, device=None, stream=None):
+
+class Workspace:
+    """Device scratch for steps of one shape (a zeroed torch uint8 buffer);
+    ``selfcond=True`` sizes it for ``denoise_step_selfcond``."""
+
+    def __init__(self, B: int, d: int, V: int, e_dtype: int = E_BF16, device=None, stream=None,
+                 selfcond: bool = False):
         import torch
-        n = workspace_size(B, d, V, e_dtype)
+        n = selfcond_workspace_size(B, d, V, e_dtype) if selfcond else workspace_size(B, d, V, e_dtype)
         if n == 0:
             raise DGError(2, "workspace_size")
         self.nbytes = n
@@ -360,6 +374,35 @@ def denoise_loop_graph(E, hidden_graph, h_buf, canvas, prev_argmax, has_prev, ac
         _ptr(stop), _ptr(state.buf), ctypes.c_size_t(state.nbytes), _ptr(ws.buf), ctypes.c_size_t(ws.nbytes),
         _stream(stream)), "dg_denoise_loop_graph")
     return steps
+
+
+def embedder_transpose(E, E_t, e_fp8: bool = False, stream=None) -> None:
+    """E_t [d, V] bf16 = E^T (``dg_embedder_transpose``); E bf16 [V, d], or
+    E4M3 codes (uint8) with ``e_fp8``."""
+    V, d = E.shape
+    shp = _shape(1, d, V, E_FP8_E4M3 if e_fp8 else E_BF16)
+    _check(lib().dg_embedder_transpose(ctypes.byref(shp), _ptr(E), _ptr(E_t), _stream(stream)),
+           "dg_embedder_transpose")
+
+
+def denoise_step_selfcond(h, E, E_t, step_idx, has_prev, canvas, prev_argmax, accept, entropy, sampled, argmax,
+                          stop, signal, ws: Workspace, params: Params = Params(), e_scale=None,
+                          stream=None) -> None:
+    """One step plus the self-conditioning signal (``dg_denoise_step_selfcond``):
+    ``signal`` float32 [B*256, d]; ``ws`` made with ``selfcond=True``."""
+    B = int(len(step_idx))
+    R, d = h.shape
+    V = E.shape[0]
+    e_dtype = E_BF16 if e_scale is None else E_FP8_E4M3
+    shp = _shape(B, d, V, e_dtype, L=R // max(B, 1))
+    prm = params.c()
+    ks = _host(step_idx, np.int32)
+    hp = _host(has_prev, np.uint8)
+    _check(lib().dg_denoise_step_selfcond(
+        ctypes.byref(shp), ctypes.byref(prm), _ptr(h), _ptr(E), _ptr(e_scale), _ptr(E_t),
+        ks.ctypes.data_as(ctypes.c_void_p), hp.ctypes.data_as(ctypes.c_void_p), _ptr(canvas), _ptr(prev_argmax),
+        _ptr(accept), _ptr(entropy), _ptr(sampled), _ptr(argmax), _ptr(stop), _ptr(signal), _ptr(ws.buf),
+        ctypes.c_size_t(ws.nbytes), _stream(stream)), "dg_denoise_step_selfcond")
 
 
 def init_canvas(canvas, B: int, V: int, params: Params = Params(), d: int = 64, stream=None) -> None:

@@ -17,6 +17,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libdg.so")
 
 SOURCES = ["dg_api.cu", "head_sampler.cu", "hidden_split.cu", "merge_select.cu", "diagnostics.cu", "noalloc.cu",
+           "selfcond.cu",
            "blocks.cu", "loop_graph.cu"]
 HEADERS = ["dg_device.cuh", "dg_internal.h", "per_device.h"]
 

@@ -137,6 +137,9 @@ struct StepArgs {
   const float* part_in = nullptr; // merge only: S shards' records [S][7][R][P]
   int32_t S = 1, P = 0;           // merge only
   const LoopDevState* loop = nullptr;  // device-side loop: per-canvas data from device memory
+  uint16_t* ptilde = nullptr;          // self-conditioning: block-scaled probabilities [R, V]
+  float* pref = nullptr;               // and their block references [R, V / 64]
+  float2* rowstat = nullptr;           // and the merged (m2, 1 / S) per row
 };
 
 // Every check of a step's arguments except those of the workspace: shape,
@@ -274,6 +277,8 @@ dg_status run_step(const StepArgs& a) {
     hp.wait_ns = kDefaultWaitNs;
     memcpy(hp.cp, cps, sizeof(cps));
 
+    hp.ptilde = a.ptilde;
+    hp.pref = a.pref;
     if (a.loop != nullptr) {
       hp.cp_dev = a.loop->cp;
       hp.mtile_dev = a.loop->canvas_of;
@@ -311,6 +316,7 @@ dg_status run_step(const StepArgs& a) {
   mp.stop_entropy = pr.stop_entropy;
   memcpy(mp.cp, cps, sizeof(cps));
   memcpy(mp.canvas_of, upd, sizeof(upd));
+  mp.rowstat = a.rowstat;
   if (a.loop != nullptr) {
     mp.cp_dev = a.loop->cp;
     mp.canvas_of_dev = a.loop->canvas_of;
@@ -338,6 +344,56 @@ dg_status enqueue_loop_step(const dg_shape* shape, const dg_params* params, cons
   return run_step(a);
 }
 
+// Self-conditioning workspace: the step's workspace, then P [R, V] bf16,
+// the block references [R, V / 64], the row statistics [R] float2 and the
+// split-K partial sums [Sk, R, d] float32.
+struct SelfcondLayout {
+  size_t p_off, pref_off, stat_off, part_off, total;
+};
+
+SelfcondLayout selfcond_layout(const dg_shape& s, size_t step_ws, int gemm_pairs) {
+  SelfcondLayout l;
+  const size_t R = static_cast<size_t>(s.B) * s.L;
+  l.p_off = align_up(step_ws);
+  l.pref_off = align_up(l.p_off + R * s.V * 2);
+  l.stat_off = align_up(l.pref_off + R * (s.V / 64) * 4);
+  l.part_off = align_up(l.stat_off + R * 8);
+  const int sk = selfcond_slices(static_cast<int>(R), s.d, s.V, gemm_pairs);
+  l.total = align_up(l.part_off + static_cast<size_t>(sk) * R * s.d * 4);
+  return l;
+}
+
+dg_status run_selfcond_step(const dg_shape* shape, const dg_params* params, const void* h, const void* E,
+                            const float* e_scale, const void* E_t, const int32_t* step_idx,
+                            const uint8_t* has_prev, int32_t* canvas, int32_t* prev_argmax, uint8_t* accept,
+                            float* entropy, int32_t* sampled, int32_t* argmax, int32_t* stop, float* signal,
+                            void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  if (E_t == nullptr || signal == nullptr || !aligned16(E_t) || !aligned16(signal)) return DG_ERR_INVALID_ARG;
+  dg_status st = check_step_call(shape, params, h, E, e_scale, step_idx, has_prev, canvas, prev_argmax, accept,
+                                 entropy, sampled, argmax, stop);
+  if (st != DG_OK) return st;
+  const size_t step_ws = dg_workspace_size(shape);
+  const int gp = selfcond_gemm_pairs();
+  if (step_ws == 0 || gp < 1) return DG_ERR_CUDA;
+  const SelfcondLayout lay = selfcond_layout(*shape, step_ws, gp);
+  if (workspace == nullptr || ws_bytes < lay.total) return DG_ERR_WORKSPACE;
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+  StepArgs a{shape,  params,  h,       E,      e_scale, step_idx, has_prev,  nullptr,  canvas, prev_argmax,
+             accept, entropy, sampled, argmax, stop,    nullptr,  workspace, step_ws, stream};
+  a.ptilde = reinterpret_cast<uint16_t*>(wsb + lay.p_off);
+  a.pref = reinterpret_cast<float*>(wsb + lay.pref_off);
+  a.rowstat = reinterpret_cast<float2*>(wsb + lay.stat_off);
+  if ((st = run_step(a)) != DG_OK) return st;
+  const int R = shape->B * shape->L;
+  if (!cuda_ok(launch_selfcond(a.ptilde, static_cast<const uint16_t*>(E_t), a.pref, a.rowstat,
+                               shape->e_dtype == DG_E_FP8_E4M3 ? e_scale : nullptr,
+                               reinterpret_cast<float*>(wsb + lay.part_off), signal, R, shape->d, shape->V,
+                               reinterpret_cast<uint32_t*>(wsb), stream),
+               "self-conditioning launch"))
+    return DG_ERR_CUDA;
+  return DG_OK;
+}
+
 dg_status check_shape_and_params(const dg_shape* shape, const dg_params* params) {
   const dg_status st = check_shape(shape);
   return st != DG_OK ? st : check_params(params);
@@ -360,11 +416,13 @@ dg_status read_and_clear_latch(void* latch, cudaStream_t st) {
   if (err != 0) {
     if (!cuda_ok(cudaMemsetAsync(latch, 0, sizeof(err), st), "fault latch clear")) return DG_ERR_CUDA;
     if (!cuda_ok(cudaStreamSynchronize(st), "stream synchronise")) return DG_ERR_CUDA;
-    if (err & ~static_cast<uint32_t>(kErrHiddenRange)) {
+    if (err & ~kErrValueMask) {
       set_last_error_message("a device-side bounded wait ran out");
       return DG_ERR_TIMEOUT;
     }
-    set_last_error_message("FP8 head: a hidden-state value is not finite");
+    set_last_error_message((err & kErrHiddenRange) ? "FP8 head: a hidden-state value is not finite"
+                                                   : "self-conditioning: logits span more than the "
+                                                     "probability blocks' range");
     return DG_ERR_VALUE;
   }
   return DG_OK;
@@ -575,6 +633,36 @@ dg_status dg_selftest_bounded_wait(uint64_t limit_ns, void* workspace, size_t ws
       cudaSuccess)
     return DG_ERR_CUDA;
   return dg_device_status(workspace, ws_bytes, stream);
+}
+
+size_t dg_selfcond_workspace_size(const dg_shape* shape) {
+  const size_t step_ws = dg_workspace_size(shape);
+  if (step_ws == 0) return 0;
+  const int gp = selfcond_gemm_pairs();
+  if (gp < 1) return 0;
+  return selfcond_layout(*shape, step_ws, gp).total;
+}
+
+dg_status dg_embedder_transpose(const dg_shape* shape, const void* E, void* E_t, void* stream) {
+  dg_status st = check_shape(shape);
+  if (st != DG_OK) return st;
+  if (E == nullptr || E_t == nullptr) return DG_ERR_INVALID_ARG;
+  if (device_sms() <= 0) return DG_ERR_NO_DEVICE;
+  if (!cuda_ok(launch_transpose(E, shape->e_dtype == DG_E_FP8_E4M3, static_cast<uint16_t*>(E_t), shape->V,
+                                shape->d, static_cast<cudaStream_t>(stream)),
+               "transpose launch"))
+    return DG_ERR_CUDA;
+  return DG_OK;
+}
+
+dg_status dg_denoise_step_selfcond(const dg_shape* shape, const dg_params* params, const void* h, const void* E,
+                                   const float* e_scale, const void* E_t, const int32_t* step_idx,
+                                   const uint8_t* has_prev, int32_t* canvas, int32_t* prev_argmax,
+                                   uint8_t* accept, float* entropy, int32_t* sampled, int32_t* argmax,
+                                   int32_t* stop, float* signal, void* workspace, size_t ws_bytes, void* stream) {
+  return run_selfcond_step(shape, params, h, E, e_scale, E_t, step_idx, has_prev, canvas, prev_argmax, accept,
+                           entropy, sampled, argmax, stop, signal, workspace, ws_bytes,
+                           static_cast<cudaStream_t>(stream));
 }
 
 dg_status dg_debug_gumbel(const uint32_t* words, int32_t n, float* g_exact, float* lg2e_approx,

@@ -23,7 +23,11 @@ enum : uint32_t {
   kErrWaitEpilogue = 1u << 3,     // epilogue gave up waiting for a finished tile
   kErrSelftest = 1u << 4,         // the bounded-wait self test ran out (expected)
   kErrHiddenRange = 1u << 5,      // FP8 head: a hidden-state value is not finite
+  kErrProbRange = 1u << 6,        // self-conditioning: a probability block outside its encoding's range
 };
+// Latched codes that report a value problem (DG_ERR_VALUE) rather than a
+// bounded wait that ran out (DG_ERR_TIMEOUT).
+constexpr uint32_t kErrValueMask = kErrHiddenRange | kErrProbRange;
 
 // ---------------------------------------------------------------------------
 // small PTX helpers

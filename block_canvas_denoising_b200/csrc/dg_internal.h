@@ -97,6 +97,11 @@ struct HeadParams {
   const CanvasParam* cp_dev;
   const uint8_t* mtile_dev;
   const int32_t* mt_dev;
+  // Self-conditioning signal: when set, also write the block-scaled
+  // probabilities ptilde[r, v] = bf16(2^(z c2 - pref[r, v / 64])) [R, V] and
+  // the block references pref [R, V / 64].
+  uint16_t* ptilde;
+  float* pref;
 };
 
 struct MergeParams {
@@ -126,6 +131,7 @@ struct MergeParams {
   const CanvasParam* cp_dev;
   const uint8_t* canvas_of_dev;
   const int32_t* n_dev;
+  float2* rowstat;  // self-conditioning: per row (m2, 1 / S) of the merged softmax, or null
 };
 
 // kblock: K elements per stage (kBlockK, or kBlockKFp8 for the FP8 head);
@@ -193,6 +199,20 @@ cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream, bool pdl = t
 // (0, s | 3 << 16, ctr_step, b): the uniform noise a block starts from.
 cudaError_t launch_init_canvas(int32_t* canvas, int B, int L, int V, uint32_t ctr_step, uint32_t seed_lo,
                                uint32_t seed_hi, cudaStream_t stream);
+// Self-conditioning signal (selfcond.cu): normalise the head's block-scaled
+// probabilities P [R, V] (bf16, in place) with the merged row statistics,
+// then signal = P . Et^T by split-K tcgen05 GEMM into `part` and a fixed-
+// order reduction.  e_scale: the FP8 embedder's row scales (folded into P),
+// else null.
+cudaError_t launch_selfcond(const uint16_t* P, const uint16_t* Et, const float* pref, const float2* rowstat,
+                            const float* e_scale, float* part, float* signal, int R, int d, int V, uint32_t* err,
+                            cudaStream_t stream);
+// K slices of the split-K GEMM and co-resident CTA pairs of it (per device).
+int selfcond_slices(int R, int d, int V, int pairs);
+int selfcond_gemm_pairs();
+// Et[c, v] = E[v, c] as bf16 (E4M3 codes widen exactly); V, d multiples of 32.
+cudaError_t launch_transpose(const void* E, bool fp8, uint16_t* Et, int V, int d, cudaStream_t stream);
+
 // The argument checks shared by the entry points (shape; parameters).
 dg_status check_shape_and_params(const dg_shape* shape, const dg_params* params);
 cudaError_t launch_wait_selftest(uint32_t* err, uint64_t limit_ns, cudaStream_t stream);

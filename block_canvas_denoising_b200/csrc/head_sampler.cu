@@ -41,6 +41,8 @@
 #include <float.h>
 #include <limits.h>
 
+#include <cuda_bf16.h>
+
 #include "dg_device.cuh"
 #include "dg_internal.h"
 #include "per_device.h"
@@ -263,10 +265,39 @@ DG_DEV void process8(const float (&z)[8], int v0, float inv_tau, float c2, const
 
 // Scales (FP8 embedder: z = (acc * s_v) * rinv, rinv = 2^-k_r), optional
 // logits dump, then the group's reductions.
+// Self-conditioning: the group's block-scaled probabilities
+// bf16(2^(z c2 - ref)) for the 64-entry block it belongs to; the block's
+// reference is set at its first group: the running maximum so far, or the
+// group's own maximum when the unit has just started (values of later
+// groups may exceed 1; a block whose values exceed 2^126 latches a fault).
+// Kept out of line: it runs only when the signal is requested, and its
+// registers must not weigh on the sampler's loop.
+__device__ __noinline__ float write_probabilities(float4 za, float4 zb, int v0, int row, float c2, const HeadParams& p,
+                                                 float m2, float blk_ref) {
+  const float z[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
+  if ((v0 & 63) == 0) {
+    const float g = fmaxf(fmaxf(fmaxf(z[0], z[1]), fmaxf(z[2], z[3])), fmaxf(fmaxf(z[4], z[5]), fmaxf(z[6], z[7])));
+    blk_ref = fmaxf(m2, g * c2);
+    p.pref[static_cast<size_t>(row) * (p.V / 64) + v0 / 64] = blk_ref;
+  }
+  uint32_t w[4];
+  bool over = false;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float d0 = fmaf(z[2 * j], c2, -blk_ref), d1 = fmaf(z[2 * j + 1], c2, -blk_ref);
+    over |= (d0 > 126.0f) || (d1 > 126.0f);
+    const __nv_bfloat162 b = __floats2bfloat162_rn(ex2_approx(fminf(d0, 126.0f)), ex2_approx(fminf(d1, 126.0f)));
+    w[j] = *reinterpret_cast<const uint32_t*>(&b);
+  }
+  if (over) atomicOr(p.err, kErrProbRange);
+  *reinterpret_cast<uint4*>(p.ptilde + static_cast<size_t>(row) * p.V + v0) = make_uint4(w[0], w[1], w[2], w[3]);
+  return blk_ref;
+}
+
 template <bool kFp8>
 DG_DEV void epi_group(const uint32_t* r, int v0, int row, float rinv, float inv_tau, float c2,
                       const PhiloxRow& pr, float thr, bool have_wm, uint32_t wm_pre, const HeadParams& p,
-                      Partial& pt, Screen& sc) {
+                      Partial& pt, Screen& sc, float& blk_ref) {
   float z[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) z[j] = __uint_as_float(r[j]);
@@ -282,6 +313,9 @@ DG_DEV void epi_group(const uint32_t* r, int v0, int row, float rinv, float inv_
     dst[0] = make_float4(z[0], z[1], z[2], z[3]);
     dst[1] = make_float4(z[4], z[5], z[6], z[7]);
   }
+  if (p.ptilde != nullptr)
+    blk_ref = write_probabilities(make_float4(z[0], z[1], z[2], z[3]), make_float4(z[4], z[5], z[6], z[7]), v0, row,
+                                  c2, p, pt.m2, blk_ref);
   // z, e_scale and the dump are indexed within this launch's rows of E; the
   // sampler (Philox counters, token indices) uses the global vocabulary index
   process8(z, v0 + p.v_off, inv_tau, c2, pr, p.rk0, p.rk1, thr, have_wm, wm_pre, pt, sc);
@@ -295,7 +329,9 @@ DG_DEV void epilogue_sync() {
 }  // namespace
 
 template <bool kFp8>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kHeadThreads, 1)
+// 576 threads x at most 112 registers fit one CTA per SM (the FP8 instance
+// needs about 106 without spilling)
+__global__ void __cluster_dims__(2, 1, 1) __maxnreg__(112)
 head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
                     const __grid_constant__ CUtensorMap tmB, const __grid_constant__ HeadParams p) {
   using Cfg = HeadCfg<kFp8>;
@@ -591,6 +627,7 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                                 key_order_dec(grec));
         grec = __ldcg(p.row_rec + row);
         uint32_t ra[8], rb[8];
+        float blk_ref = 0.f;  // self-conditioning: this tile's 64-entry block reference
         __syncwarp();
         tmem_load8_issue(tbase, ra);
         tmem_load8_wait(ra);
@@ -598,11 +635,11 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         for (int g = 0; g < kGroups; g += 2) {
           tmem_load8_issue(tbase + 8 * (g + 1), rb);
           epi_group<kFp8>(ra, vbase + 8 * g, row, rinv, inv_tau, c2, pr, thr, mma_quarter,
-                          mma_quarter ? wsrc[g * 32] : 0u, p, pt, sc);
+                          mma_quarter ? wsrc[g * 32] : 0u, p, pt, sc, blk_ref);
           tmem_load8_wait(rb);
           if (g + 2 < kGroups) tmem_load8_issue(tbase + 8 * (g + 2), ra);
           epi_group<kFp8>(rb, vbase + 8 * (g + 1), row, rinv, inv_tau, c2, pr, thr, mma_quarter,
-                          mma_quarter ? wsrc[(g + 1) * 32] : 0u, p, pt, sc);
+                          mma_quarter ? wsrc[(g + 1) * 32] : 0u, p, pt, sc, blk_ref);
           tmem_load8_wait(ra);
           __syncwarp();
         }

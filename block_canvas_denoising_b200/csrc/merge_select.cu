@@ -105,6 +105,7 @@ merge_select_kernel(const __grid_constant__ MergeParams p) {
     double H = log1p(sp) - 0.69314718055994530942 * static_cast<double>(a.T2) / (1.0 + sp);
     H = H > 0.0 ? H : 0.0;
     p.entropy[row] = static_cast<float>(H);
+    if (p.rowstat != nullptr) p.rowstat[row] = make_float2(a.m2, static_cast<float>(1.0 / (1.0 + sp)));
     p.sampled[row] = a.garg;
     p.argmax[row] = a.zarg;
   }

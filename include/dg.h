@@ -181,7 +181,8 @@ dg_status dg_debug_logits(const dg_shape* shape, const dg_params* params,
 
 /* Synchronise `stream`, then read and clear the device fault latch of the
  * workspace.  Returns DG_OK, DG_ERR_TIMEOUT (a bounded wait ran out),
- * DG_ERR_VALUE (FP8 head: a non-finite h) or DG_ERR_CUDA. */
+ * DG_ERR_VALUE (FP8 head: a non-finite h; self-conditioning: logits beyond
+ * the probability encoding's range) or DG_ERR_CUDA. */
 dg_status dg_device_status(void* workspace, size_t ws_bytes, void* stream);
 
 /* Hidden-state producer for the loop: writes the bf16 [B*L, d] hidden
@@ -218,6 +219,45 @@ dg_status dg_denoise_loop(const dg_shape* shape, const dg_params* params,
                           uint8_t* accept, float* entropy, int32_t* sampled,
                           int32_t* argmax, int32_t* stop,
                           void* workspace, size_t ws_bytes, void* stream);
+
+/* ---- self-conditioning signal ([Report] Table 1: a 7.8M-parameter MLP
+ * "for self-conditioning"; the pages define neither the signal nor the
+ * MLP).  Reading: the signal of slot r is the embedding expected under the
+ * step's tempered distribution, s[r] = sum_v softmax(z[r] / tau_k)_v E[v]
+ * (a d-vector per slot), the input such an MLP would project.  The MLP has
+ * trained weights and is out of scope.
+ *
+ * The head writes block-scaled bf16 probabilities while it samples, a pass
+ * normalises them with the merged softmax statistics, and a split-K tcgen05
+ * GEMM against E^T (both operands K-major) with a fixed-order reduction
+ * forms s.  P is rounded to bf16 twice (block-scaled, then normalised):
+ * |s_gpu - s| <= 2^-8 sum_v p_v |E[v]| per element, plus float32 sums. */
+
+/* E_t = E^T as bf16 [d, V] row-major (device, d * V * 2 bytes, caller-
+ * owned): E's bf16 values, or for the FP8 embedder its E4M3 codes widened
+ * to bf16 exactly (the row scales are applied to the probabilities).  Made
+ * once per embedder. */
+dg_status dg_embedder_transpose(const dg_shape* shape, const void* E, void* E_t, void* stream);
+
+/* Workspace bytes of dg_denoise_step_selfcond on the current device: the
+ * step's workspace, P (B*L*V bf16), the block references, the row
+ * statistics and the split-K partial sums.  0 for an invalid shape. */
+size_t dg_selfcond_workspace_size(const dg_shape* shape);
+
+/* dg_denoise_step_selfcond -- dg_denoise_step (every canvas updated; no
+ * `active`) that also writes the self-conditioning signal
+ *   signal  float [B*L, d] (device, 16-byte aligned).
+ * E_t from dg_embedder_transpose of the same E; workspace of
+ * dg_selfcond_workspace_size() bytes (zeroed once, like a step's).  A
+ * block of logits spanning more than the bf16 probability encoding can hold
+ * (2^126) latches DG_ERR_VALUE (see dg_device_status). */
+dg_status dg_denoise_step_selfcond(const dg_shape* shape, const dg_params* params,
+                                   const void* h, const void* E, const float* e_scale, const void* E_t,
+                                   const int32_t* step_idx, const uint8_t* has_prev,
+                                   int32_t* canvas, int32_t* prev_argmax,
+                                   uint8_t* accept, float* entropy, int32_t* sampled,
+                                   int32_t* argmax, int32_t* stop, float* signal,
+                                   void* workspace, size_t ws_bytes, void* stream);
 
 /* ---- the adaptive loop on the device -------------------------------------
  * dg_denoise_loop reads the stop flags back to the host after every step.

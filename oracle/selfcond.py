@@ -22,11 +22,14 @@ from .step import decode_bf16, decode_e4m3, logits, temperature
 
 
 def expected_embedding(h_bits, *, E_bits=None, q=None, s=None, k: int, tau0: float = 0.8, tau1: float = 0.4,
-                       max_steps: int = 48, v_chunk: int = 8192) -> np.ndarray:
+                       max_steps: int = 48, v_chunk: int = 8192, abs_values: bool = False) -> np.ndarray:
     """s = softmax(z / tau_k) @ E in float64, [rows, d]; the embedder given
     as bf16 bits or as E4M3 codes q with row scales s.  Two passes over the
     vocabulary: the row maxima of x = z / tau, then the weighted sum of the
-    rows of E with weights e^{x - max} and the normaliser."""
+    rows of E with weights e^{x - max} and the normaliser.  With
+    ``abs_values`` the weighted sum is over |E| (same weights): the scale
+    sum_v p_v |E[v]| that bounds the error of a signal computed with
+    rounded weights."""
     tau = temperature(k, tau0, tau1, max_steps)
     z = logits(h_bits, E_bits=E_bits, q=q, s=s)
     x = z / tau
@@ -41,5 +44,7 @@ def expected_embedding(h_bits, *, E_bits=None, q=None, s=None, k: int, tau0: flo
             Ec = decode_bf16(E_bits[v0:v1])
         else:
             Ec = decode_e4m3(q[v0:v1]) * np.asarray(s[v0:v1], dtype=np.float64)[:, None]
+        if abs_values:
+            Ec = np.abs(Ec)
         out += w[:, v0:v1] @ Ec
     return out / w.sum(axis=1, keepdims=True)

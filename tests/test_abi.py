@@ -182,3 +182,23 @@ def test_device_loop_host_checks(libdg):
     assert call(nbytes=n1 - 1) == 3
     assert call(hpv=None) == 1
     assert call(prm=dg.Params(max_steps=0)) == 1
+
+
+def test_selfcond_host_checks(libdg):
+    # E_t and signal are required and 16-byte aligned; the workspace must
+    # hold the signal's scratch (refused before any device work)
+    shp = dg._Shape(1, 256, 512, 4096, 0)
+    prm = dg.Params().c()
+    ks = np.zeros(1, np.int32)
+    hp = np.zeros(1, np.uint8)
+    fake = ctypes.c_void_p(4096)
+    kp, hpp = ks.ctypes.data_as(ctypes.c_void_p), hp.ctypes.data_as(ctypes.c_void_p)
+
+    def call(E_t=fake, signal=fake):
+        return libdg.dg_denoise_step_selfcond(ctypes.byref(shp), ctypes.byref(prm), fake, fake, None, E_t, kp, hpp,
+                                              *([fake] * 7), signal, fake, ctypes.c_size_t(1 << 40), None)
+    assert call(E_t=None) == 1
+    assert call(signal=ctypes.c_void_p(4100)) == 1
+    assert libdg.dg_embedder_transpose(ctypes.byref(dg._Shape(1, 128, 512, 4096, 0)), fake, fake, None) == 2
+    assert libdg.dg_embedder_transpose(ctypes.byref(shp), None, fake, None) == 1
+    assert libdg.dg_selfcond_workspace_size(ctypes.byref(dg._Shape(1, 256, 100, 4096, 0))) == 0

@@ -72,3 +72,17 @@ def test_fp8_embedder_uses_the_dequantised_rows():
     p = np.exp(x - x.max(axis=1, keepdims=True))
     p /= p.sum(axis=1, keepdims=True)
     assert np.allclose(got, p @ Ed, rtol=0, atol=1e-15)
+
+
+def test_abs_values_scale_bounds_the_signal():
+    # sum_v p_v |E[v]| >= |sum_v p_v E[v]| elementwise, with equality where
+    # E's column has one sign; for a non-negative embedder the two agree
+    V, d = 512, 32
+    E = synth.embedder_normal(V, d, seed=4)
+    h = synth.hidden_normal(1, 4, d, seed=5)
+    s_ = selfcond.expected_embedding(h, E_bits=E, k=3)
+    a_ = selfcond.expected_embedding(h, E_bits=E, k=3, abs_values=True)
+    assert np.all(a_ >= np.abs(s_) - 1e-15) and np.any(a_ > np.abs(s_) + 1e-6)
+    Epos = (np.asarray(E, np.uint16) & np.uint16(0x7FFF)).astype(np.uint16)
+    assert np.allclose(selfcond.expected_embedding(h, E_bits=Epos, k=3),
+                       selfcond.expected_embedding(h, E_bits=Epos, k=3, abs_values=True), rtol=0, atol=1e-15)
