@@ -67,6 +67,8 @@ def parse():
     ap.add_argument("--e-dtype", default="bf16", choices=("bf16", "fp8"))
     ap.add_argument("--batch", type=int, default=1, help="canvases per GPU per step")
     ap.add_argument("--no-loop", action="store_true", help="skip the untimed production-shape loop run")
+    ap.add_argument("--selfcond", action="store_true",
+                    help="also time the step with the self-conditioning signal (expected embedding)")
     return ap.parse_args()
 
 
@@ -372,25 +374,34 @@ def main():
                         params, e_scale=e_scale)
 
     def timed_region(K):
-        ev_h = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in range(K)]
-        for a, b in ev_h:       # torch creates the event handles on first record
-            a.record(stream)
-            b.record(stream)
+        """K steps timed end to end with nothing else in the stream (the
+        step-throughput pass), then K steps with CUDA events recorded around
+        every fused head kernel (the kernel-time pass: an event between the
+        head and the merge keeps the merge from launching early, so it is
+        kept out of the first pass)."""
         t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
         t0.record(stream)
         for i in range(K):
-            dg.set_head_events(*ev_h[i])
             step(i, h)
-        dg.set_head_events(None, None)
         t1.record(stream)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         total_ms = t0.elapsed_time(t1)
+        ev_h = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(K)]
+        for a, b in ev_h:       # torch creates the event handles on first record
+            a.record(stream)
+            b.record(stream)
+        torch.cuda.synchronize()
+        for i in range(K):
+            dg.set_head_events(*ev_h[i])
+            step(i, h)
+        dg.set_head_events(None, None)
+        torch.cuda.synchronize()
         head_ms = sum(a.elapsed_time(b) for a, b in ev_h) / K
         return total_ms, head_ms
 
@@ -461,6 +472,47 @@ def main():
     e2e_ms = e2e_total / K2
     e2e_value = world * B * L / (e2e_ms / 1e3)
 
+    sc_line = None
+    if args.selfcond:
+        # the step with the self-conditioning signal s = softmax(z / tau) E:
+        # head (+ block-scaled probabilities), merge, normalisation, split-K
+        # GEMM against E^T, reduction; timed the same way
+        E_t = torch.empty((D, V), dtype=torch.bfloat16, device="cuda")
+        dg.embedder_transpose(E, E_t, e_fp8=fp8)
+        ws_sc = dg.Workspace(B, D, V, ws_dtype, selfcond=True)
+        signal = torch.empty((R, D), dtype=torch.float32, device="cuda")
+
+        def sc_step(i):
+            dg.denoise_step_selfcond(h, E, E_t, ks_of[i % len(ks_of)], hp_rest if i > 0 else hp_first,
+                                     dev["canvas"], dev["prev"], dev["acc"], dev["ent"], dev["samp"], dev["amax"],
+                                     dev["stop"], signal, ws_sc, params, e_scale=e_scale)
+        for i in range(max(3, args.warmup)):
+            sc_step(i)
+        torch.cuda.synchronize()
+        K3 = max(3, args.steps)
+        if world > 1:
+            dist.barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for i in range(K3):
+            sc_step(i)
+        s1.record(stream)
+        torch.cuda.synchronize()
+        assert dg.device_status(ws_sc) == 0
+        (sc_total,) = reduce_max([s0.elapsed_time(s1)], dist, "cuda")
+        sc_ms = sc_total / K3
+        pk, _ = peaks()
+        # the signal's own roofline: one more stream of E (as E^T) and
+        # 2 R d V flops
+        sc_roof_us = max(V * D * 2 / (pk["hbm_gbs"] * 1e9), 2.0 * R * D * V / (pk["bf16_tflops"] * 1e12)) * 1e6
+        extra_us = (sc_ms - ms_per_step) * 1e3
+        sc_line = {"us_per_step": sc_ms * 1e3, "extra_us_over_step": extra_us,
+                   "signal_roofline_us": sc_roof_us, "signal_frac": sc_roof_us / extra_us if extra_us > 0 else None,
+                   "what": "step + expected-embedding signal [B*256, d] float32 (P bf16 written by the head, "
+                           "normalised, split-K tcgen05 GEMM against E^T, fixed-order reduction)",
+                   "gpu_launches_per_step": (3 if fp8 else 2) + 3}
+        del ws_sc, E_t
+
     loop = None
     if world == 1 and not args.no_loop:
         loop = loop_report(dg, E, E_bits, e_scale, fp8, ws_dtype, torch, B)
@@ -513,9 +565,13 @@ def main():
             "e2e": {"value": e2e_value, "unit": "slots/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": (3 if fp8 else 2) * args.steps,
+            "timing": "ms_per_step from K steps with no events in the stream; roofline.kernel_us from a second "
+                      "pass of K steps with events around each fused head kernel",
         }
         if loop is not None:
             line["loop"] = loop
+        if sc_line is not None:
+            line["selfcond"] = sc_line
         if world == 1 and B == 1 and not args.no_cpu_baseline and not fp8:
             t_cpu = oracle_canvas_step(h_bits, E_bits, 0)
             line["cpu_baseline"] = {"value": L / t_cpu, "unit": "slots/s", "cores": threads_used(),

@@ -286,7 +286,8 @@ dg_status run_step(const StepArgs& a) {
     }
     const bool events = t_head_ev_start != nullptr && a.loop == nullptr;
     if (events && cudaEventRecord(t_head_ev_start, a.stream) != cudaSuccess) return DG_ERR_CUDA;
-    if (!cuda_ok(launch_head(fp8, tmA, tmA2, tmB, hp, a.stream), "head kernel launch")) return DG_ERR_CUDA;
+    if (!cuda_ok(launch_head(fp8, tmA, tmA2, tmB, hp, a.stream, a.loop == nullptr), "head kernel launch"))
+      return DG_ERR_CUDA;
     if (events && cudaEventRecord(t_head_ev_stop, a.stream) != cudaSuccess) return DG_ERR_CUDA;
   }
   if (!merge) return DG_OK;

@@ -185,8 +185,10 @@ dg_status read_and_clear_latch(void* latch, cudaStream_t st);
 
 // bf16 head: tmA = h bf16 [R, d], tmB = E bf16 [V, d] (tmA2 unused).
 // FP8 head:  tmA = h1, tmA2 = h2 (E4M3 [R, d]), tmB = E codes E4M3 [V, d].
+// pdl: launch as a programmatic dependent of the preceding kernel (off
+// inside graphs built by the device-side loop).
 cudaError_t launch_head(bool fp8, const CUtensorMap& tmA, const CUtensorMap& tmA2, const CUtensorMap& tmB,
-                        const HeadParams& p, cudaStream_t stream);
+                        const HeadParams& p, cudaStream_t stream, bool pdl = true);
 // Split each row r of h (bf16 [R, d], d a multiple of 8, 16-byte aligned)
 // into E4M3 terms h1 + h2 = h * 2^k_r and write rinv[r] = 2^-k_r; latches
 // kErrHiddenRange in *err if some h is not finite.

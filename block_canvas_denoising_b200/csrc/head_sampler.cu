@@ -52,22 +52,35 @@ namespace dg {
 namespace {
 
 // Row tiles this launch covers, and the per-canvas data: from device memory
-// in the device-side loop, else from the launch parameters.
-DG_DEV int row_tiles(const HeadParams& p) { return p.mt_dev != nullptr ? __ldcg(p.mt_dev) : p.split.MT; }
+// in the device-side loop's instance (kDev), else from the launch
+// parameters (a separate instance keeps those reads out of the sampler's
+// register budget).
+template <bool kDev>
+DG_DEV int row_tiles(const HeadParams& p) {
+  if constexpr (kDev) return __ldcg(p.mt_dev);
+  return p.split.MT;
+}
+template <bool kDev>
 DG_DEV CanvasParam canvas_param(const HeadParams& p, int b) {
-  if (p.cp_dev == nullptr) return p.cp[b];
-  CanvasParam c;
-  c.k = __ldcg(&p.cp_dev[b].k);
-  c.inv_tau = __ldcg(&p.cp_dev[b].inv_tau);
-  return c;
+  if constexpr (kDev) {
+    CanvasParam c;
+    c.k = __ldcg(&p.cp_dev[b].k);
+    c.inv_tau = __ldcg(&p.cp_dev[b].inv_tau);
+    return c;
+  }
+  return p.cp[b];
 }
 
 // Unit u: row tile (canvas) m, vocabulary tiles [n0, n1), unit index q
 // within the row tile; mt = row_tiles(p).
+template <bool kDev>
 DG_DEV void unit_range(const HeadParams& p, int mt, int u, int& m, int& n0, int& n1, int& q) {
   const HeadSplit& sp = p.split;
   q = u / mt;
-  m = p.mtile_dev != nullptr ? static_cast<int>(__ldcg(p.mtile_dev + (u - q * mt))) : p.mtile[u - q * mt];
+  if constexpr (kDev)
+    m = static_cast<int>(__ldcg(p.mtile_dev + (u - q * mt)));
+  else
+    m = p.mtile[u - q * mt];
   n0 = static_cast<int>((static_cast<int64_t>(q) * sp.NT) / sp.Q);
   n1 = static_cast<int>((static_cast<int64_t>(q + 1) * sp.NT) / sp.Q);
 }
@@ -126,13 +139,36 @@ DG_DEV void top2(float& a1, float& a2, float b1, float b2) {
   a1 = hi;
 }
 
+// The Philox counter words of one slot, (slot | purpose << 16, k, b): with
+// kHoist the first two rounds' slot-constant products formed once
+// (philox_row), else the three words themselves (the FP8 instance, whose
+// registers are tighter, draws with the plain rounds).
+template <bool kHoist>
+DG_DEV PhiloxRow slot_counter(uint32_t c1, uint32_t c2, uint32_t c3, const uint32_t (&rk0)[10],
+                              const uint32_t (&rk1)[10]) {
+  if constexpr (kHoist) return philox_row(c1, c2, c3, rk0, rk1);
+  PhiloxRow r;
+  r.x0r1 = c1;
+  r.b1 = c2;
+  r.e0 = c3;
+  r.c1k = 0;
+  r.d = 0;
+  return r;
+}
+
 // The Philox words of the 8 consecutive vocabulary entries 4 cb .. 4 cb + 7
-// of the slot whose row constants are `pr`.
+// of the slot whose counter words are `pr`.
+template <bool kHoist>
 DG_DEV void philox_words8(uint32_t cb, const PhiloxRow& pr, const uint32_t (&rk0)[10], const uint32_t (&rk1)[10],
                           uint32_t (&w)[8]) {
   uint32_t wa[4], wb[4];
-  philox4x32_10_row(cb, pr, rk0, rk1, wa);
-  philox4x32_10_row(cb + 1, pr, rk0, rk1, wb);
+  if constexpr (kHoist) {
+    philox4x32_10_row(cb, pr, rk0, rk1, wa);
+    philox4x32_10_row(cb + 1, pr, rk0, rk1, wb);
+  } else {
+    philox4x32_10_keys(cb, pr.x0r1, pr.b1, pr.e0, rk0, rk1, wa);
+    philox4x32_10_keys(cb + 1, pr.x0r1, pr.b1, pr.e0, rk0, rk1, wb);
+  }
 #pragma unroll
   for (int l = 0; l < 4; ++l) {
     w[l] = wa[l];
@@ -146,6 +182,7 @@ DG_DEV void philox_words8(uint32_t cb, const PhiloxRow& pr, const uint32_t (&rk0
 // wm_pre: when have_wm (warp-uniform), the group's largest Philox word,
 // computed beforehand by another warp; the words themselves are then drawn
 // here only if the group passes its bound.
+template <bool kHoist>
 DG_DEV void process8(const float (&z)[8], int v0, float inv_tau, float c2, const PhiloxRow& pr,
                      const uint32_t (&rk0)[10], const uint32_t (&rk1)[10], float thr, bool have_wm,
                      uint32_t wm_pre, Partial& pt, Screen& sc) {
@@ -219,9 +256,9 @@ DG_DEV void process8(const float (&z)[8], int v0, float inv_tau, float c2, const
   uint32_t w[8];
   if (have_wm) {
     if (__fmaf_rn(lg2_exp1_approx(wm_pre), -kLn2, x0max) < lim_eps) return;
-    philox_words8(cb, pr, rk0, rk1, w);
+    philox_words8<kHoist>(cb, pr, rk0, rk1, w);
   } else {
-    philox_words8(cb, pr, rk0, rk1, w);
+    philox_words8<kHoist>(cb, pr, rk0, rk1, w);
     const uint32_t wm = max(max(max(w[0], w[1]), max(w[2], w[3])), max(max(w[4], w[5]), max(w[6], w[7])));
     if (__fmaf_rn(lg2_exp1_approx(wm), -kLn2, x0max) < lim_eps) return;
   }
@@ -294,7 +331,7 @@ __device__ __noinline__ float write_probabilities(float4 za, float4 zb, int v0, 
   return blk_ref;
 }
 
-template <bool kFp8>
+template <bool kFp8, bool kProbs>
 DG_DEV void epi_group(const uint32_t* r, int v0, int row, float rinv, float inv_tau, float c2,
                       const PhiloxRow& pr, float thr, bool have_wm, uint32_t wm_pre, const HeadParams& p,
                       Partial& pt, Screen& sc, float& blk_ref) {
@@ -313,12 +350,12 @@ DG_DEV void epi_group(const uint32_t* r, int v0, int row, float rinv, float inv_
     dst[0] = make_float4(z[0], z[1], z[2], z[3]);
     dst[1] = make_float4(z[4], z[5], z[6], z[7]);
   }
-  if (p.ptilde != nullptr)
+  if (kProbs)
     blk_ref = write_probabilities(make_float4(z[0], z[1], z[2], z[3]), make_float4(z[4], z[5], z[6], z[7]), v0, row,
                                   c2, p, pt.m2, blk_ref);
   // z, e_scale and the dump are indexed within this launch's rows of E; the
   // sampler (Philox counters, token indices) uses the global vocabulary index
-  process8(z, v0 + p.v_off, inv_tau, c2, pr, p.rk0, p.rk1, thr, have_wm, wm_pre, pt, sc);
+  process8<!kFp8>(z, v0 + p.v_off, inv_tau, c2, pr, p.rk0, p.rk1, thr, have_wm, wm_pre, pt, sc);
 }
 
 // Named barrier over the epilogue warps only (barrier 1).
@@ -328,10 +365,15 @@ DG_DEV void epilogue_sync() {
 
 }  // namespace
 
-template <bool kFp8>
-// 576 threads x at most 112 registers fit one CTA per SM (the FP8 instance
-// needs about 106 without spilling)
-__global__ void __cluster_dims__(2, 1, 1) __maxnreg__(112)
+// One CTA of 576 threads per SM: its 18 warps share the four schedulers'
+// register files as 5 + 5 + 4 + 4 warps, so a thread may use at most 96
+// registers (5 x 32 x 96 <= 16,384), which the launch bound enforces.
+// kProbs: the self-conditioning instance, which also writes the block-scaled
+// probabilities; kDev: the device-side loop's instance, which reads the
+// per-canvas data from device memory (separate instances keep that code out
+// of the plain sampler's register budget).
+template <bool kFp8, bool kProbs, bool kDev>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kHeadThreads, 1)
 head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
                     const __grid_constant__ CUtensorMap tmB, const __grid_constant__ HeadParams p) {
   using Cfg = HeadCfg<kFp8>;
@@ -359,7 +401,7 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   const int pair = blockIdx.x >> 1;
   const int npairs = gridDim.x >> 1;
   const HeadSplit& sp = p.split;
-  const int mt = row_tiles(p);       // row tiles (canvases) of this launch
+  const int mt = row_tiles<kDev>(p);       // row tiles (canvases) of this launch
   const int units = mt * sp.Q;
 
   auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
@@ -395,6 +437,11 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Launched as a programmatic dependent of the preceding kernel (the
+  // previous step's merge, which clears the key records and reads the
+  // partial records this launch overwrites): the set-up above overlaps its
+  // tail; nothing here reads or writes global memory before it completes.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
@@ -409,7 +456,7 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       bool ok = true;
       for (int u = pair; u < units && ok; u += npairs) {
         int m, n0, n1, q;
-        unit_range(p, mt, u, m, n0, n1, q);
+        unit_range<kDev>(p, mt, u, m, n0, n1, q);
         for (int n = n0; n < n1 && ok; ++n) {
           for (int kb = 0; kb < sp.KB; ++kb) {
             if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, p.wait_ns)) {
@@ -468,7 +515,7 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       bool ok = true;
       for (int u = pair; u < units && ok; u += npairs) {
         int m, n0, n1, q;
-        unit_range(p, mt, u, m, n0, n1, q);
+        unit_range<kDev>(p, mt, u, m, n0, n1, q);
         for (int n = n0; n < n1 && ok; ++n, ++tile) {
           const int acc = tile & 1;
           const uint32_t acc_phase = (tile >> 1) & 1;
@@ -543,10 +590,10 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         const int hrow = m_t * kPairM + static_cast<int>(rank) * kBlockM + kMmaQuarter * 32 + r;
         const int hb = hrow >> 8;
         uint32_t w[8];
-        const PhiloxRow pr = philox_row(static_cast<uint32_t>(hrow & 255) | (kPurposeGumbel << 16),
-                                        static_cast<uint32_t>(canvas_param(p, hb).k), static_cast<uint32_t>(hb), p.rk0,
-                                        p.rk1);
-        philox_words8(static_cast<uint32_t>(p.v_off + n_t * kBlockN + g * 8) >> 2, pr, p.rk0, p.rk1, w);
+        const PhiloxRow pr = slot_counter<!kFp8>(static_cast<uint32_t>(hrow & 255) | (kPurposeGumbel << 16),
+                                                 static_cast<uint32_t>(canvas_param<kDev>(p, hb).k),
+                                                 static_cast<uint32_t>(hb), p.rk0, p.rk1);
+        philox_words8<!kFp8>(static_cast<uint32_t>(p.v_off + n_t * kBlockN + g * 8) >> 2, pr, p.rk0, p.rk1, w);
         dst[g * 32 + r] = max(max(max(w[0], w[1]), max(w[2], w[3])), max(max(w[4], w[5]), max(w[6], w[7])));
       }
       __syncwarp();
@@ -559,22 +606,22 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     bool ok = true;
     if (!mma_quarter && pair < units) {
       int m, n0, n1, q;
-      unit_range(p, mt, pair, m, n0, n1, q);
+      unit_range<kDev>(p, mt, pair, m, n0, n1, q);
       ok = produce_words(0, m, n0);
     }
     for (int u = pair; u < units; u += npairs) {
       int m, n0, n1, q;
-      unit_range(p, mt, u, m, n0, n1, q);
+      unit_range<kDev>(p, mt, u, m, n0, n1, q);
       const int row = m * kPairM + static_cast<int>(rank) * kBlockM + rloc;
       const int b = row >> 8;
       const int slot = row & 255;
-      const CanvasParam cp = canvas_param(p, b);
+      const CanvasParam cp = canvas_param<kDev>(p, b);
       const float inv_tau = cp.inv_tau;
       const float rinv = kFp8 ? __ldg(p.row_inv + row) : 1.0f;
       const float c2 = __fmul_rn(inv_tau, kLog2e);
       // Philox counter (v >> 2, slot | purpose << 16, k, b): the row's constants
-      const PhiloxRow pr = philox_row(static_cast<uint32_t>(slot) | (kPurposeGumbel << 16),
-                                      static_cast<uint32_t>(cp.k), static_cast<uint32_t>(b), p.rk0, p.rk1);
+      const PhiloxRow pr = slot_counter<!kFp8>(static_cast<uint32_t>(slot) | (kPurposeGumbel << 16),
+                                               static_cast<uint32_t>(cp.k), static_cast<uint32_t>(b), p.rk0, p.rk1);
       Partial pt;
       partial_init(pt);
       Screen sc;
@@ -592,7 +639,7 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           bool more = nn < n1;
           if (!more && u + npairs < units) {
             int n1n, qn;
-            unit_range(p, mt, u + npairs, mn, nn, n1n, qn);
+            unit_range<kDev>(p, mt, u + npairs, mn, nn, n1n, qn);
             more = true;
           }
           if (more && !produce_words(tile + 1, mn, nn)) {
@@ -634,11 +681,11 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 #pragma unroll 1
         for (int g = 0; g < kGroups; g += 2) {
           tmem_load8_issue(tbase + 8 * (g + 1), rb);
-          epi_group<kFp8>(ra, vbase + 8 * g, row, rinv, inv_tau, c2, pr, thr, mma_quarter,
+          epi_group<kFp8, kProbs>(ra, vbase + 8 * g, row, rinv, inv_tau, c2, pr, thr, mma_quarter,
                           mma_quarter ? wsrc[g * 32] : 0u, p, pt, sc, blk_ref);
           tmem_load8_wait(rb);
           if (g + 2 < kGroups) tmem_load8_issue(tbase + 8 * (g + 2), ra);
-          epi_group<kFp8>(rb, vbase + 8 * (g + 1), row, rinv, inv_tau, c2, pr, thr, mma_quarter,
+          epi_group<kFp8, kProbs>(rb, vbase + 8 * (g + 1), row, rinv, inv_tau, c2, pr, thr, mma_quarter,
                           mma_quarter ? wsrc[(g + 1) * 32] : 0u, p, pt, sc, blk_ref);
           tmem_load8_wait(ra);
           __syncwarp();
@@ -721,10 +768,10 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 
 // Launch set-up of one head variant on the current device: allow its
 // dynamic shared memory, then count the CTA pairs that fit at once.
-template <bool kFp8>
+template <bool kFp8, bool kProbs, bool kDev>
 bool setup_on_current_device(int* pairs) {
   constexpr int kSmem = HeadCfg<kFp8>::kSmemBytes;
-  if (cudaFuncSetAttribute(head_sampler_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) !=
+  if (cudaFuncSetAttribute(head_sampler_kernel<kFp8, kProbs, kDev>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) !=
       cudaSuccess)
     return false;
   cudaLaunchConfig_t cfg = {};
@@ -739,23 +786,26 @@ bool setup_on_current_device(int* pairs) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, head_sampler_kernel<kFp8>, &cfg) != cudaSuccess || n < 1) return false;
+  if (cudaOccupancyMaxActiveClusters(&n, head_sampler_kernel<kFp8, kProbs, kDev>, &cfg) != cudaSuccess || n < 1)
+    return false;
   *pairs = n;
   return true;
 }
 
 // Co-resident CTA pairs of a head variant on the current device (-1 if it
 // cannot run there), set up once per device.
-template <bool kFp8>
+template <bool kFp8, bool kProbs, bool kDev>
 int max_pairs_of() {
   static PerDevice<int> cache;
   int dev = -1, pairs = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return -1;
-  if (!cache.get(dev, [](int* v) { return setup_on_current_device<kFp8>(v); }, &pairs)) return -1;
+  if (!cache.get(dev, [](int* v) { return setup_on_current_device<kFp8, kProbs, kDev>(v); }, &pairs)) return -1;
   return pairs;
 }
 
-int head_max_pairs(bool fp8) { return fp8 ? max_pairs_of<true>() : max_pairs_of<false>(); }
+// The sampler instances decide the work split; the self-conditioning
+// instances must fit the same number of pairs (checked at launch).
+int head_max_pairs(bool fp8) { return fp8 ? max_pairs_of<true, false, false>() : max_pairs_of<false, false, false>(); }
 
 HeadSplit head_split(int R, int V, int d, int max_pairs, int kblock, int q_cap) {
   HeadSplit s;
@@ -779,14 +829,38 @@ HeadSplit head_split(int R, int V, int d, int max_pairs, int kblock, int q_cap) 
 }
 
 cudaError_t launch_head(bool fp8, const CUtensorMap& tmA, const CUtensorMap& tmA2, const CUtensorMap& tmB,
-                        const HeadParams& p, cudaStream_t stream) {
-  if (head_max_pairs(fp8) < 1) return cudaErrorInvalidConfiguration;
-  if (fp8)
-    head_sampler_kernel<true><<<p.split.grid, kHeadThreads, HeadCfg<true>::kSmemBytes, stream>>>(tmA, tmA2, tmB, p);
+                        const HeadParams& p, cudaStream_t stream, bool pdl) {
+  const bool probs = p.ptilde != nullptr;
+  const bool dev = p.cp_dev != nullptr;
+  if (probs && dev) return cudaErrorInvalidValue;  // no instance writes the signal inside the device loop
+  int fit;
+  if (probs)
+    fit = fp8 ? max_pairs_of<true, true, false>() : max_pairs_of<false, true, false>();
+  else if (dev)
+    fit = fp8 ? max_pairs_of<true, false, true>() : max_pairs_of<false, false, true>();
   else
-    head_sampler_kernel<false><<<p.split.grid, kHeadThreads, HeadCfg<false>::kSmemBytes, stream>>>(tmA, tmA2, tmB,
-                                                                                                    p);
-  return cudaGetLastError();
+    fit = head_max_pairs(fp8);
+  if (fit < p.split.grid / 2) return cudaErrorInvalidConfiguration;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.split.grid, 1, 1);
+  cfg.blockDim = dim3(kHeadThreads, 1, 1);
+  cfg.dynamicSmemBytes = fp8 ? HeadCfg<true>::kSmemBytes : HeadCfg<false>::kSmemBytes;
+  cfg.stream = stream;
+  // programmatic dependent launch: the set-up overlaps the preceding
+  // kernel's tail; griddepcontrol.wait in the kernel orders the data
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  if (fp8) {
+    if (probs) return cudaLaunchKernelEx(&cfg, head_sampler_kernel<true, true, false>, tmA, tmA2, tmB, p);
+    if (dev) return cudaLaunchKernelEx(&cfg, head_sampler_kernel<true, false, true>, tmA, tmA2, tmB, p);
+    return cudaLaunchKernelEx(&cfg, head_sampler_kernel<true, false, false>, tmA, tmA2, tmB, p);
+  }
+  if (probs) return cudaLaunchKernelEx(&cfg, head_sampler_kernel<false, true, false>, tmA, tmA2, tmB, p);
+  if (dev) return cudaLaunchKernelEx(&cfg, head_sampler_kernel<false, false, true>, tmA, tmA2, tmB, p);
+  return cudaLaunchKernelEx(&cfg, head_sampler_kernel<false, false, false>, tmA, tmA2, tmB, p);
 }
 
 }  // namespace dg

@@ -79,8 +79,10 @@ merge_select_kernel(const __grid_constant__ MergeParams p) {
   const int row = b * 256 + (blockIdx.x % kCtasPerCanvas) * kRowsPerCta + warp;
   const size_t plane = static_cast<size_t>(p.R) * p.P;
 
-  // Launched as a programmatic dependent of the head kernel: wait until its
-  // partial records are complete and visible.
+  // The next step's head may launch now (it waits for this grid before it
+  // touches memory); then wait, as a programmatic dependent of the head,
+  // until the partial records are complete and visible.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // ---- merge the P partial records of this row: lane j takes j, j+32, ...;
