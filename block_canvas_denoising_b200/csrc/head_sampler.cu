@@ -813,7 +813,13 @@ HeadSplit head_split(int R, int V, int d, int max_pairs, int kblock, int q_cap) 
   s.NT = V / kBlockN;
   s.KB = (d + kblock - 1) / kblock;
   const long long quads = static_cast<long long>(s.MT) * (s.NT / 4);
-  if (s.NT % 4 == 0 && quads >= 8LL * max_pairs) {
+  const long long octs = static_cast<long long>(s.MT) * (s.NT / 8);
+  if (s.NT % 8 == 0 && octs >= 8LL * max_pairs) {
+    // units of 8 vocabulary tiles, many per pair (fewer unit ends: each
+    // merges the column groups' records and meets two named barriers;
+    // measured 1.2 % faster than units of 4 at B = 32)
+    s.Q = s.NT / 8;
+  } else if (s.NT % 4 == 0 && quads >= 8LL * max_pairs) {
     s.Q = s.NT / 4;  // units of 4 vocabulary tiles, many per pair
   } else {
     int q = max_pairs / s.MT;
