@@ -98,8 +98,8 @@ struct HeadParams {
   const uint8_t* mtile_dev;
   const int32_t* mt_dev;
   // Self-conditioning signal: when set, also write the block-scaled
-  // probabilities ptilde[r, v] = bf16(2^(z c2 - pref[r, v / 64])) [R, V] and
-  // the block references pref [R, V / 64].
+  // probabilities ptilde[r, v] = bf16(2^(z c2 - pref[v / 64, r])) [R, V] and
+  // the block references pref [V / 64, R].
   uint16_t* ptilde;
   float* pref;
 };

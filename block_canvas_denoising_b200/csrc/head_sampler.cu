@@ -307,15 +307,14 @@ DG_DEV void process8(const float (&z)[8], int v0, float inv_tau, float c2, const
 // reference is set at its first group: the running maximum so far, or the
 // group's own maximum when the unit has just started (values of later
 // groups may exceed 1; a block whose values exceed 2^126 latches a fault).
-// Kept out of line: it runs only when the signal is requested, and its
-// registers must not weigh on the sampler's loop.
-__device__ __noinline__ float write_probabilities(float4 za, float4 zb, int v0, int row, float c2, const HeadParams& p,
+// Only the self-conditioning instances (kProbs) contain it.
+__device__ __forceinline__ float write_probabilities(float4 za, float4 zb, int v0, int row, float c2, const HeadParams& p,
                                                  float m2, float blk_ref) {
   const float z[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
   if ((v0 & 63) == 0) {
     const float g = fmaxf(fmaxf(fmaxf(z[0], z[1]), fmaxf(z[2], z[3])), fmaxf(fmaxf(z[4], z[5]), fmaxf(z[6], z[7])));
     blk_ref = fmaxf(m2, g * c2);
-    p.pref[static_cast<size_t>(row) * (p.V / 64) + v0 / 64] = blk_ref;
+    p.pref[static_cast<size_t>(v0 / 64) * p.R + row] = blk_ref;  // [V / 64][R]: coalesced over rows
   }
   uint32_t w[4];
   bool over = false;
@@ -814,10 +813,13 @@ HeadSplit head_split(int R, int V, int d, int max_pairs, int kblock, int q_cap) 
   s.KB = (d + kblock - 1) / kblock;
   const long long quads = static_cast<long long>(s.MT) * (s.NT / 4);
   const long long octs = static_cast<long long>(s.MT) * (s.NT / 8);
-  if (s.NT % 8 == 0 && octs >= 8LL * max_pairs) {
-    // units of 8 vocabulary tiles, many per pair (fewer unit ends: each
-    // merges the column groups' records and meets two named barriers;
-    // measured 1.2 % faster than units of 4 at B = 32)
+  const long long hexs = static_cast<long long>(s.MT) * (s.NT / 16);
+  // The longest units that still give every pair at least 8: fewer unit ends
+  // (each merges the column groups' records and meets two named barriers).
+  // Measured at B = 32: units of 8 tiles 1.2 % faster than 4, 16 another 0.9 %.
+  if (s.NT % 16 == 0 && hexs >= 8LL * max_pairs) {
+    s.Q = s.NT / 16;
+  } else if (s.NT % 8 == 0 && octs >= 8LL * max_pairs) {
     s.Q = s.NT / 8;
   } else if (s.NT % 4 == 0 && quads >= 8LL * max_pairs) {
     s.Q = s.NT / 4;  // units of 4 vocabulary tiles, many per pair

@@ -14,14 +14,18 @@
 //      scaled probabilities: Pt[r, v] = bf16(2^(z c2 - ref)) for each block
 //      of 64 vocabulary entries with its own reference ref[r, block] (the
 //      running maximum when the block starts), ref to `pref`;
-//   2. normalise (here): P[r, v] = bf16(Pt[r, v] 2^(ref - m2_r) / S_r) in
-//      place, with the row's final maximum m2_r and normaliser S_r from the
-//      merge (and the FP8 embedder's row scale s_v folded in);
+//   2. normalise: P[r, v] = bf16(Pt[r, v] 2^(ref - m2_r) / S_r), with the
+//      row's final maximum m2_r and normaliser S_r from the merge -- for the
+//      bf16 embedder inside the GEMM (transform warps scale each row of a
+//      landed P tile in shared memory before the MMA reads it: one factor per
+//      row and 64-entry block, which is exactly one K stage), for the FP8
+//      embedder in a separate pass that also folds in the row scales s_v;
 //   3. split-K GEMM (here, tcgen05 pairs): partial[q] = P[:, K_q] . Et[:, K_q]^T
 //      over vocabulary slices K_q, with Et = E^T [d, V] bf16 made once per
 //      embedder (dg_embedder_transpose), so both operands are K-major;
 //   4. reduce (here): s = sum_q partial[q] in a fixed order.
 #include <cudaTypedefs.h>
+#include <cuda_bf16.h>
 #include <cuda_fp8.h>
 #include <string.h>
 
@@ -38,7 +42,9 @@ namespace {
 // ---------------------------------------------------------------------------
 constexpr int kGemmStages = 6;
 constexpr int kGemmEpiWarps = 8;                       // 4 lane quarters x 2 column halves
-constexpr int kGemmThreads = (2 + kGemmEpiWarps) * 32;
+constexpr int kGemmXfWarps = 4;                        // transform: one P row per thread (128 rows)
+constexpr int kGemmXfWarp0 = 2 + kGemmEpiWarps;
+constexpr int kGemmThreads = (2 + kGemmEpiWarps + kGemmXfWarps) * 32;
 constexpr int kGemmSmem = kGemmStages * 2 * kTileBytes + 1024 + 256;
 static_assert(kGemmSmem <= 232448, "split-K GEMM exceeds 227 KB of shared memory");
 
@@ -49,6 +55,10 @@ struct GemmParams {
   float* part;             // [Sk][R][d]
   uint32_t* err;
   uint64_t wait_ns;
+  // kScale: the transform warps scale row r of stage kb by
+  // 2^(pref[kb, r] - rowstat[r].x) * rowstat[r].y
+  const float* pref;       // [V / 64][R]
+  const float2* rowstat;   // [R] (m2, 1 / S)
 };
 
 // Unit u: d tile n (fastest, so pairs running at once share the P slice in
@@ -62,6 +72,13 @@ DG_DEV void gemm_unit(const GemmParams& p, int u, int& m, int& n, int& q, int& k
   k1 = static_cast<int>((static_cast<int64_t>(q + 1) * p.KB) / p.Sk);
 }
 
+// kScale: P arrives block-scaled (the head's Pt) and the transform warps
+// normalise each landed A tile in shared memory; the MMA then waits for the
+// tile to be both landed and scaled (`ready`, arrivals of both CTAs'
+// transform warps).  Without it the A tiles are already normalised and the
+// MMA waits for them to land (`full`, the leader's barrier with both CTAs'
+// bytes).
+template <bool kScale>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 selfcond_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ GemmParams p) {
@@ -70,7 +87,8 @@ selfcond_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
   uint8_t* sA = smem;
   uint8_t* sB = smem + kGemmStages * kTileBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sB + kGemmStages * kTileBytes);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kGemmStages + 4);
+  // barriers: full[S], empty[S], tfull[2], tempty[2], ready[S]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * kGemmStages + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -81,6 +99,7 @@ selfcond_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
   auto empty_bar = [&](int s) { return smem_u32(&bars[kGemmStages + s]); };
   auto tfull_bar = [&](int a) { return smem_u32(&bars[2 * kGemmStages + a]); };
   auto tempty_bar = [&](int a) { return smem_u32(&bars[2 * kGemmStages + 2 + a]); };
+  auto ready_bar = [&](int s) { return smem_u32(&bars[2 * kGemmStages + 4 + s]); };
 
   if (threadIdx.x == 0) {
     prefetch_tensormap(&tmA);
@@ -93,6 +112,7 @@ selfcond_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       mbar_init(tfull_bar(a), 1);
       mbar_init(tempty_bar(a), 2 * kGemmEpiWarps);
     }
+    for (int s = 0; s < kGemmStages; ++s) mbar_init(ready_bar(s), 2 * kGemmXfWarps);
     fence_mbarrier_init();
   }
   if (warp == 0) {
@@ -121,12 +141,19 @@ selfcond_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             break;
           }
           const uint32_t fb = full_bar(stage);
-          if (rank == 0) mbar_arrive_expect_tx(fb, 4 * kTileBytes);
-          const uint32_t fb_leader = mapa_shared(fb, 0);
+          uint32_t fb_dst;
+          if (kScale) {
+            // this CTA's transform warps wait for its own tiles
+            mbar_arrive_expect_tx(fb, 2 * kTileBytes);
+            fb_dst = mapa_shared(fb, rank);
+          } else {
+            if (rank == 0) mbar_arrive_expect_tx(fb, 4 * kTileBytes);
+            fb_dst = mapa_shared(fb, 0);
+          }
           const int kx = kb * kBlockK;
-          tma_load_2d_pair(smem_u32(sA + stage * kTileBytes), &tmA, fb_leader, kx,
+          tma_load_2d_pair(smem_u32(sA + stage * kTileBytes), &tmA, fb_dst, kx,
                            m * kPairM + static_cast<int>(rank) * kBlockM, pol);
-          tma_load_2d_pair(smem_u32(sB + stage * kTileBytes), &tmB, fb_leader, kx,
+          tma_load_2d_pair(smem_u32(sB + stage * kTileBytes), &tmB, fb_dst, kx,
                            n * kBlockN + static_cast<int>(rank) * kHalfN, pol);
           if (++stage == kGemmStages) {
             stage = 0;
@@ -169,7 +196,9 @@ selfcond_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBlockN);
         for (int kb = k0; kb < k1; ++kb) {
-          if (!mbar_wait_bounded(full_bar(stage), phase, p.wait_ns)) {
+          const bool landed = kScale ? mbar_wait_bounded<true>(ready_bar(stage), phase, p.wait_ns)
+                                     : mbar_wait_bounded(full_bar(stage), phase, p.wait_ns);
+          if (!landed) {
             atomicOr(p.err, kErrWaitMmaFull);
             ok = false;
             break;
@@ -188,6 +217,59 @@ selfcond_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
           }
         }
         if (ok) tc_commit_pair_mc(tfull_bar(acc), 0x3);
+      }
+    }
+  } else if (warp >= kGemmXfWarp0) {
+    // ---- transform (kScale): thread t scales row t of this CTA's A tile of
+    // each landed stage; a K stage is one 64-entry probability block, so the
+    // row has one factor (the 128-byte swizzle only permutes 16-byte chunks
+    // within the row)
+    if (kScale) {
+      const int t = threadIdx.x - kGemmXfWarp0 * 32;
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int u = pair; u < p.units; u += npairs) {
+        int m, n, q, k0, k1;
+        gemm_unit(p, u, m, n, q, k0, k1);
+        const int row = m * kPairM + static_cast<int>(rank) * kBlockM + t;
+        const float2 st = __ldg(p.rowstat + row);
+        for (int kb = k0; kb < k1; ++kb) {
+          const float ref = __ldg(p.pref + static_cast<size_t>(kb) * p.R + row);
+          const float f = exp2f(ref - st.x) * st.y;
+          if (ok && !mbar_wait_bounded(full_bar(stage), phase, p.wait_ns)) {
+            atomicOr(p.err, kErrWaitEpilogue);
+            ok = false;
+          }
+          if (ok) {
+            uint4* rp = reinterpret_cast<uint4*>(sA + stage * kTileBytes + t * 128);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              uint4 w = rp[c];
+              uint32_t* wp = &w.x;
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const __nv_bfloat162 o =
+                    __floats2bfloat162_rn(__uint_as_float(wp[j] << 16) * f, __uint_as_float(wp[j] & 0xFFFF0000u) * f);
+                wp[j] = *reinterpret_cast<const uint32_t*>(&o);
+              }
+              rp[c] = w;
+            }
+            // the tensor core reads the tile through the async proxy
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) {
+              if (rank == 0)
+                mbar_arrive(ready_bar(stage));
+              else
+                mbar_arrive_remote(mapa_shared(ready_bar(stage), 0));
+            }
+          }
+          if (++stage == kGemmStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
       }
     }
   } else {
@@ -241,8 +323,9 @@ selfcond_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
   }
 }
 
+template <bool kScale>
 bool gemm_setup(int* pairs) {
-  if (cudaFuncSetAttribute(selfcond_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem) !=
+  if (cudaFuncSetAttribute(selfcond_gemm_kernel<kScale>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem) !=
       cudaSuccess)
     return false;
   cudaLaunchConfig_t cfg = {};
@@ -257,9 +340,18 @@ bool gemm_setup(int* pairs) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, selfcond_gemm_kernel, &cfg) != cudaSuccess || n < 1) return false;
+  if (cudaOccupancyMaxActiveClusters(&n, selfcond_gemm_kernel<kScale>, &cfg) != cudaSuccess || n < 1) return false;
   *pairs = n;
   return true;
+}
+
+template <bool kScale>
+int gemm_pairs_of() {
+  static PerDevice<int> cache;
+  int dev = -1, pairs = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (!cache.get(dev, [](int* v) { return gemm_setup<kScale>(v); }, &pairs)) return -1;
+  return pairs;
 }
 
 // ---------------------------------------------------------------------------
@@ -274,7 +366,7 @@ __global__ void __launch_bounds__(256) selfcond_normalize_kernel(uint4* __restri
   const int r = static_cast<int>(i / v8);
   const int v0 = static_cast<int>(i - static_cast<size_t>(r) * v8) * 8;
   const float2 st = __ldg(rowstat + r);  // (m2, 1 / S)
-  const float ref = __ldg(pref + static_cast<size_t>(r) * (V / 64) + v0 / 64);
+  const float ref = __ldg(pref + static_cast<size_t>(v0 / 64) * R + r);
   const float f = exp2f(ref - st.x) * st.y;
   uint4 w = pt[i];
   uint32_t* wp = &w.x;
@@ -362,13 +454,8 @@ bool encode_kmajor(CUtensorMap* map, const void* base, uint64_t inner, uint64_t 
 
 }  // namespace
 
-int selfcond_gemm_pairs() {
-  static PerDevice<int> cache;
-  int dev = -1, pairs = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
-  if (!cache.get(dev, [](int* v) { return gemm_setup(v); }, &pairs)) return -1;
-  return pairs;
-}
+// The split used for both instances (they fit the same pairs; checked at launch).
+int selfcond_gemm_pairs() { return gemm_pairs_of<false>(); }
 
 int selfcond_slices(int R, int d, int V, int pairs) {
   const int MT = R / kPairM, NT = (d + kBlockN - 1) / kBlockN, KB = V / kBlockK;
@@ -383,13 +470,16 @@ cudaError_t launch_selfcond(const uint16_t* P, const uint16_t* Et, const float* 
                             cudaStream_t stream) {
   const int pairs = selfcond_gemm_pairs();
   if (pairs < 1) return cudaErrorInvalidConfiguration;
-  // 2. normalise
-  const size_t n8 = static_cast<size_t>(R) * (V / 8);
-  selfcond_normalize_kernel<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, stream>>>(
-      reinterpret_cast<uint4*>(const_cast<uint16_t*>(P)), pref, rowstat, e_scale, R, V);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  // 3. split-K GEMM
+  const bool scale_in_gemm = e_scale == nullptr;  // bf16: one factor per row and K stage
+  cudaError_t e;
+  if (!scale_in_gemm) {
+    // 2. normalise in place, folding in the FP8 row scales (a factor per element)
+    const size_t n8 = static_cast<size_t>(R) * (V / 8);
+    selfcond_normalize_kernel<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, stream>>>(
+        reinterpret_cast<uint4*>(const_cast<uint16_t*>(P)), pref, rowstat, e_scale, R, V);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  // 3. split-K GEMM (with the normalisation of the bf16 case inside)
   CUtensorMap tmA, tmB;
   if (!encode_kmajor(&tmA, P, V, R, kBlockM) || !encode_kmajor(&tmB, Et, V, d, kHalfN))
     return cudaErrorInvalidValue;
@@ -406,8 +496,14 @@ cudaError_t launch_selfcond(const uint16_t* P, const uint16_t* Et, const float* 
   gp.part = part;
   gp.err = err;
   gp.wait_ns = kDefaultWaitNs;
-  const int grid = 2 * (gp.units < pairs ? gp.units : pairs);
-  selfcond_gemm_kernel<<<grid, kGemmThreads, kGemmSmem, stream>>>(tmA, tmB, gp);
+  gp.pref = pref;
+  gp.rowstat = rowstat;
+  const int use = gp.units < pairs ? gp.units : pairs;
+  if ((scale_in_gemm ? gemm_pairs_of<true>() : pairs) < use) return cudaErrorInvalidConfiguration;
+  if (scale_in_gemm)
+    selfcond_gemm_kernel<true><<<2 * use, kGemmThreads, kGemmSmem, stream>>>(tmA, tmB, gp);
+  else
+    selfcond_gemm_kernel<false><<<2 * use, kGemmThreads, kGemmSmem, stream>>>(tmA, tmB, gp);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // 4. reduce
   const size_t n4 = static_cast<size_t>(R) * d / 4;

@@ -348,7 +348,7 @@ dg_status dg_generate_blocks(const dg_shape* shape, const dg_params* params,
  * exits.  Shapes needing more (dg_workspace_size() > 8 MiB) return
  * DG_ERR_WORKSPACE before anything is launched, with the sizes in
  * dg_last_error_message(); on a 148-SM B200 at d = 2816, V = 262,144 that
- * is B > 9 canvases with the bf16 embedder and B > 2 with the FP8 embedder
+ * is B > 18 canvases with the bf16 embedder and B > 2 with the FP8 embedder
  * (whose scratch also holds the two E4M3 terms of h).  All argument checks
  * run before the array is touched.  The first call on a device looks the
  * array's device address up once (the runtime may initialise the context
