@@ -14,12 +14,12 @@
 //      scaled probabilities: Pt[r, v] = bf16(2^(z c2 - ref)) for each block
 //      of 64 vocabulary entries with its own reference ref[r, block] (the
 //      running maximum when the block starts), ref to `pref`;
-//   2. normalise: P[r, v] = bf16(Pt[r, v] 2^(ref - m2_r) / S_r), with the
-//      row's final maximum m2_r and normaliser S_r from the merge -- for the
-//      bf16 embedder inside the GEMM (transform warps scale each row of a
-//      landed P tile in shared memory before the MMA reads it: one factor per
-//      row and 64-entry block, which is exactly one K stage), for the FP8
-//      embedder in a separate pass that also folds in the row scales s_v;
+//   2. normalise: P[r, v] = bf16(Pt[r, v] 2^(ref - m2_r) / S_r [s_v]), with
+//      the row's final maximum m2_r and normaliser S_r from the merge (and
+//      the FP8 embedder's row scales s_v), inside the GEMM: transform warps
+//      scale each row of a landed P tile in shared memory before the MMA
+//      reads it (one factor per row and 64-entry block, which is exactly one
+//      K stage);
 //   3. split-K GEMM (here, tcgen05 pairs): partial[q] = P[:, K_q] . Et[:, K_q]^T
 //      over vocabulary slices K_q, with Et = E^T [d, V] bf16 made once per
 //      embedder (dg_embedder_transpose), so both operands are K-major;
@@ -55,10 +55,11 @@ struct GemmParams {
   float* part;             // [Sk][R][d]
   uint32_t* err;
   uint64_t wait_ns;
-  // kScale: the transform warps scale row r of stage kb by
-  // 2^(pref[kb, r] - rowstat[r].x) * rowstat[r].y
+  // the transform warps scale row r of stage kb by
+  // 2^(pref[kb, r] - rowstat[r].x) * rowstat[r].y (times s_v for FP8)
   const float* pref;       // [V / 64][R]
   const float2* rowstat;   // [R] (m2, 1 / S)
+  const float* e_scale;    // FP8 embedder: per-vocabulary-row scales folded into P, else null
 };
 
 // Unit u: d tile n (fastest, so pairs running at once share the P slice in
@@ -72,13 +73,10 @@ DG_DEV void gemm_unit(const GemmParams& p, int u, int& m, int& n, int& q, int& k
   k1 = static_cast<int>((static_cast<int64_t>(q + 1) * p.KB) / p.Sk);
 }
 
-// kScale: P arrives block-scaled (the head's Pt) and the transform warps
-// normalise each landed A tile in shared memory; the MMA then waits for the
-// tile to be both landed and scaled (`ready`, arrivals of both CTAs'
-// transform warps).  Without it the A tiles are already normalised and the
-// MMA waits for them to land (`full`, the leader's barrier with both CTAs'
-// bytes).
-template <bool kScale>
+// P arrives block-scaled (the head's Pt) and the transform warps normalise
+// each landed A tile in shared memory; each CTA's loads complete on its own
+// `full` barrier, and the MMA waits for the stage to be both landed and
+// scaled in both CTAs (`ready`, arrivals of both CTAs' transform warps).
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 selfcond_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ GemmParams p) {
@@ -140,16 +138,10 @@ selfcond_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             ok = false;
             break;
           }
+          // this CTA's transform warps wait for its own tiles
           const uint32_t fb = full_bar(stage);
-          uint32_t fb_dst;
-          if (kScale) {
-            // this CTA's transform warps wait for its own tiles
-            mbar_arrive_expect_tx(fb, 2 * kTileBytes);
-            fb_dst = mapa_shared(fb, rank);
-          } else {
-            if (rank == 0) mbar_arrive_expect_tx(fb, 4 * kTileBytes);
-            fb_dst = mapa_shared(fb, 0);
-          }
+          mbar_arrive_expect_tx(fb, 2 * kTileBytes);
+          const uint32_t fb_dst = mapa_shared(fb, rank);
           const int kx = kb * kBlockK;
           tma_load_2d_pair(smem_u32(sA + stage * kTileBytes), &tmA, fb_dst, kx,
                            m * kPairM + static_cast<int>(rank) * kBlockM, pol);
@@ -196,9 +188,7 @@ selfcond_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBlockN);
         for (int kb = k0; kb < k1; ++kb) {
-          const bool landed = kScale ? mbar_wait_bounded<true>(ready_bar(stage), phase, p.wait_ns)
-                                     : mbar_wait_bounded(full_bar(stage), phase, p.wait_ns);
-          if (!landed) {
+          if (!mbar_wait_bounded<true>(ready_bar(stage), phase, p.wait_ns)) {
             atomicOr(p.err, kErrWaitMmaFull);
             ok = false;
             break;
@@ -220,11 +210,11 @@ selfcond_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       }
     }
   } else if (warp >= kGemmXfWarp0) {
-    // ---- transform (kScale): thread t scales row t of this CTA's A tile of
-    // each landed stage; a K stage is one 64-entry probability block, so the
-    // row has one factor (the 128-byte swizzle only permutes 16-byte chunks
+    // ---- transform: thread t scales row t of this CTA's A tile of each
+    // landed stage; a K stage is one 64-entry probability block, so the row
+    // has one factor (the 128-byte swizzle only permutes 16-byte chunks
     // within the row)
-    if (kScale) {
+    {
       const int t = threadIdx.x - kGemmXfWarp0 * 32;
       int stage = 0;
       uint32_t phase = 0;
@@ -245,12 +235,21 @@ selfcond_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             uint4* rp = reinterpret_cast<uint4*>(sA + stage * kTileBytes + t * 128);
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
+              // FP8 embedder: the row scales s_v of this chunk's 8 entries;
+              // the 128-byte swizzle stores logical chunk c ^ (t % 8) here
+              float sv[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
+              if (p.e_scale != nullptr) {
+                const float4* sp = reinterpret_cast<const float4*>(p.e_scale + kb * kBlockK + ((c ^ (t & 7)) << 3));
+                const float4 s0 = __ldg(sp), s1 = __ldg(sp + 1);
+                sv[0] = s0.x; sv[1] = s0.y; sv[2] = s0.z; sv[3] = s0.w;
+                sv[4] = s1.x; sv[5] = s1.y; sv[6] = s1.z; sv[7] = s1.w;
+              }
               uint4 w = rp[c];
               uint32_t* wp = &w.x;
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
-                const __nv_bfloat162 o =
-                    __floats2bfloat162_rn(__uint_as_float(wp[j] << 16) * f, __uint_as_float(wp[j] & 0xFFFF0000u) * f);
+                const __nv_bfloat162 o = __floats2bfloat162_rn(__uint_as_float(wp[j] << 16) * f * sv[2 * j],
+                                                               __uint_as_float(wp[j] & 0xFFFF0000u) * f * sv[2 * j + 1]);
                 wp[j] = *reinterpret_cast<const uint32_t*>(&o);
               }
               rp[c] = w;
@@ -323,9 +322,8 @@ selfcond_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
   }
 }
 
-template <bool kScale>
 bool gemm_setup(int* pairs) {
-  if (cudaFuncSetAttribute(selfcond_gemm_kernel<kScale>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem) !=
+  if (cudaFuncSetAttribute(selfcond_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem) !=
       cudaSuccess)
     return false;
   cudaLaunchConfig_t cfg = {};
@@ -340,53 +338,17 @@ bool gemm_setup(int* pairs) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, selfcond_gemm_kernel<kScale>, &cfg) != cudaSuccess || n < 1) return false;
+  if (cudaOccupancyMaxActiveClusters(&n, selfcond_gemm_kernel, &cfg) != cudaSuccess || n < 1) return false;
   *pairs = n;
   return true;
 }
 
-template <bool kScale>
 int gemm_pairs_of() {
   static PerDevice<int> cache;
   int dev = -1, pairs = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return -1;
-  if (!cache.get(dev, [](int* v) { return gemm_setup<kScale>(v); }, &pairs)) return -1;
+  if (!cache.get(dev, [](int* v) { return gemm_setup(v); }, &pairs)) return -1;
   return pairs;
-}
-
-// ---------------------------------------------------------------------------
-// normalise the block-scaled probabilities in place
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) selfcond_normalize_kernel(uint4* __restrict__ pt, const float* __restrict__ pref,
-                                                                 const float2* __restrict__ rowstat,
-                                                                 const float* __restrict__ e_scale, int R, int V) {
-  const int v8 = V / 8;
-  const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= static_cast<size_t>(R) * v8) return;
-  const int r = static_cast<int>(i / v8);
-  const int v0 = static_cast<int>(i - static_cast<size_t>(r) * v8) * 8;
-  const float2 st = __ldg(rowstat + r);  // (m2, 1 / S)
-  const float ref = __ldg(pref + static_cast<size_t>(v0 / 64) * R + r);
-  const float f = exp2f(ref - st.x) * st.y;
-  uint4 w = pt[i];
-  uint32_t* wp = &w.x;
-  float sv[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) sv[j] = 1.0f;
-  if (e_scale != nullptr) {
-    const float4 a = __ldg(reinterpret_cast<const float4*>(e_scale + v0));
-    const float4 b = __ldg(reinterpret_cast<const float4*>(e_scale + v0) + 1);
-    sv[0] = a.x; sv[1] = a.y; sv[2] = a.z; sv[3] = a.w;
-    sv[4] = b.x; sv[5] = b.y; sv[6] = b.z; sv[7] = b.w;
-  }
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const float lo = __uint_as_float(wp[j] << 16) * f * sv[2 * j];
-    const float hi = __uint_as_float(wp[j] & 0xFFFF0000u) * f * sv[2 * j + 1];
-    const __nv_bfloat162 o = __floats2bfloat162_rn(lo, hi);
-    wp[j] = *reinterpret_cast<const uint32_t*>(&o);
-  }
-  pt[i] = w;
 }
 
 // ---------------------------------------------------------------------------
@@ -454,8 +416,7 @@ bool encode_kmajor(CUtensorMap* map, const void* base, uint64_t inner, uint64_t 
 
 }  // namespace
 
-// The split used for both instances (they fit the same pairs; checked at launch).
-int selfcond_gemm_pairs() { return gemm_pairs_of<false>(); }
+int selfcond_gemm_pairs() { return gemm_pairs_of(); }
 
 int selfcond_slices(int R, int d, int V, int pairs) {
   const int MT = R / kPairM, NT = (d + kBlockN - 1) / kBlockN, KB = V / kBlockK;
@@ -470,16 +431,8 @@ cudaError_t launch_selfcond(const uint16_t* P, const uint16_t* Et, const float* 
                             cudaStream_t stream) {
   const int pairs = selfcond_gemm_pairs();
   if (pairs < 1) return cudaErrorInvalidConfiguration;
-  const bool scale_in_gemm = e_scale == nullptr;  // bf16: one factor per row and K stage
   cudaError_t e;
-  if (!scale_in_gemm) {
-    // 2. normalise in place, folding in the FP8 row scales (a factor per element)
-    const size_t n8 = static_cast<size_t>(R) * (V / 8);
-    selfcond_normalize_kernel<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, stream>>>(
-        reinterpret_cast<uint4*>(const_cast<uint16_t*>(P)), pref, rowstat, e_scale, R, V);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
-  // 3. split-K GEMM (with the normalisation of the bf16 case inside)
+  // 2 + 3. normalisation inside the split-K GEMM
   CUtensorMap tmA, tmB;
   if (!encode_kmajor(&tmA, P, V, R, kBlockM) || !encode_kmajor(&tmB, Et, V, d, kHalfN))
     return cudaErrorInvalidValue;
@@ -498,12 +451,9 @@ cudaError_t launch_selfcond(const uint16_t* P, const uint16_t* Et, const float* 
   gp.wait_ns = kDefaultWaitNs;
   gp.pref = pref;
   gp.rowstat = rowstat;
+  gp.e_scale = e_scale;
   const int use = gp.units < pairs ? gp.units : pairs;
-  if ((scale_in_gemm ? gemm_pairs_of<true>() : pairs) < use) return cudaErrorInvalidConfiguration;
-  if (scale_in_gemm)
-    selfcond_gemm_kernel<true><<<2 * use, kGemmThreads, kGemmSmem, stream>>>(tmA, tmB, gp);
-  else
-    selfcond_gemm_kernel<false><<<2 * use, kGemmThreads, kGemmSmem, stream>>>(tmA, tmB, gp);
+  selfcond_gemm_kernel<<<2 * use, kGemmThreads, kGemmSmem, stream>>>(tmA, tmB, gp);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // 4. reduce
   const size_t n4 = static_cast<size_t>(R) * d / 4;

@@ -227,10 +227,10 @@ dg_status dg_denoise_loop(const dg_shape* shape, const dg_params* params,
  * (a d-vector per slot), the input such an MLP would project.  The MLP has
  * trained weights and is out of scope.
  *
- * The head writes block-scaled bf16 probabilities while it samples, a pass
- * normalises them with the merged softmax statistics, and a split-K tcgen05
- * GEMM against E^T (both operands K-major) with a fixed-order reduction
- * forms s.  P is rounded to bf16 twice (block-scaled, then normalised):
+ * The head writes block-scaled bf16 probabilities while it samples; a
+ * split-K tcgen05 GEMM against E^T (both operands K-major) normalises each
+ * landed tile with the merged softmax statistics before multiplying, and a
+ * fixed-order reduction forms s.  P is rounded to bf16 twice (block-scaled, then normalised):
  * |s_gpu - s| <= 2^-8 sum_v p_v |E[v]| per element, plus float32 sums. */
 
 /* E_t = E^T as bf16 [d, V] row-major (device, d * V * 2 bytes, caller-
