@@ -235,16 +235,20 @@ selfcond_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             uint4* rp = reinterpret_cast<uint4*>(sA + stage * kTileBytes + t * 128);
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
-              // FP8 embedder: the row scales s_v of this chunk's 8 entries;
-              // the 128-byte swizzle stores logical chunk c ^ (t % 8) here
+              // Logical chunk c (entries 8c .. 8c + 7 of the block) sits at
+              // 16-byte slot c ^ (t % 8) under the 128-byte swizzle; visiting
+              // the row in that order puts the lanes of a warp on different
+              // banks (row by row, the same slot would be one bank group)
+              const int slot = c ^ (t & 7);
+              // FP8 embedder: the row scales s_v of the chunk's 8 entries
               float sv[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
               if (p.e_scale != nullptr) {
-                const float4* sp = reinterpret_cast<const float4*>(p.e_scale + kb * kBlockK + ((c ^ (t & 7)) << 3));
+                const float4* sp = reinterpret_cast<const float4*>(p.e_scale + kb * kBlockK + c * 8);
                 const float4 s0 = __ldg(sp), s1 = __ldg(sp + 1);
                 sv[0] = s0.x; sv[1] = s0.y; sv[2] = s0.z; sv[3] = s0.w;
                 sv[4] = s1.x; sv[5] = s1.y; sv[6] = s1.z; sv[7] = s1.w;
               }
-              uint4 w = rp[c];
+              uint4 w = rp[slot];
               uint32_t* wp = &w.x;
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
@@ -252,7 +256,7 @@ selfcond_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                                                                __uint_as_float(wp[j] & 0xFFFF0000u) * f * sv[2 * j + 1]);
                 wp[j] = *reinterpret_cast<const uint32_t*>(&o);
               }
-              rp[c] = w;
+              rp[slot] = w;
             }
             // the tensor core reads the tile through the async proxy
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -1,4 +1,5 @@
-"""The adaptive loop run on the device (``dg_denoise_loop_graph``).
+"""The adaptive loop run on the device (``dg_denoise_loop_graph``), and the
+fault path of both loops.
 
 One CUDA graph with a conditional (while) node runs every step: the
 hidden-state graph (here a torch-captured graph that copies step k's stand-in
@@ -185,3 +186,38 @@ def test_device_loop_production_shape():
     gh = _run_host(E, table, 1, d, V, params, **kw)
     _same(gd, gh)
     assert gd["steps"][0] == 3 and (gd["canvas"] == y).mean() > 0.99
+
+
+@pytest.mark.parametrize("device_loop", [False, True])
+def test_loop_stops_on_a_latched_fault(device_loop):
+    # the fault is made on the host: the workspace's fault word is set before
+    # the loop starts (no kernel faults, traps or hangs).  Both loops run one
+    # step, see the latch, stop and return the latched status; nothing was
+    # committed
+    B, d, V = 2, 256, 1024
+    E_bits = synth.embedder_normal(V, d, seed=1)
+    E = to_dev_bf16(E_bits)
+    y = synth.loop_targets(L, V, seed=3, B=B)
+    R = B * L
+    h_buf = to_dev_bf16(synth.loop_hidden(2, y, E_bits, seed=4)).contiguous()
+    canvas0 = synth.canvas_uniform(B, L, V, seed=0)
+    canvas = torch.from_numpy(canvas0.copy()).cuda()
+    prev = torch.zeros(R, dtype=torch.int32, device="cuda")
+    hp = np.zeros(B, np.uint8)
+    outs = _outs(B)
+    ws = dg.Workspace(B, d, V)
+    ws.buf[:4].view(torch.int32).fill_(1 << 2)      # a bounded wait that "ran out"
+    torch.cuda.synchronize()
+    with pytest.raises(dg.DGError) as ei:
+        if device_loop:
+            dg.denoise_loop_graph(E, None, h_buf, canvas, prev, hp, outs["accept"], outs["entropy"],
+                                  outs["sampled"], outs["argmax"], outs["stop"], ws, dg.LoopState(B), dg.Params())
+        else:
+            dg.denoise_loop(E, lambda k, c, h: None, h_buf, canvas, prev, hp, outs["accept"], outs["entropy"],
+                            outs["sampled"], outs["argmax"], outs["stop"], ws, dg.Params())
+    assert ei.value.code == 6                         # DG_ERR_TIMEOUT
+    assert dg.device_status(ws) == 0                  # reported once, then cleared
+    torch.cuda.synchronize()
+    # one step ran (the outputs are written) but no canvas was committed
+    assert int(outs["accept"].sum()) >= B
+    assert not np.array_equal(canvas.cpu().numpy(), canvas0)   # renoised by the step, not committed
