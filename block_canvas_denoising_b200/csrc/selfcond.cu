@@ -45,7 +45,8 @@ constexpr int kGemmEpiWarps = 8;                       // 4 lane quarters x 2 co
 constexpr int kGemmXfWarps = 4;                        // transform: one P row per thread (128 rows)
 constexpr int kGemmXfWarp0 = 2 + kGemmEpiWarps;
 constexpr int kGemmThreads = (2 + kGemmEpiWarps + kGemmXfWarps) * 32;
-constexpr int kGemmSmem = kGemmStages * 2 * kTileBytes + 1024 + 256;
+constexpr int kRefBytes = kBlockM * 4;  // a stage's block references of this CTA's 128 rows
+constexpr int kGemmSmem = kGemmStages * (2 * kTileBytes + kRefBytes) + 1024 + 256;
 static_assert(kGemmSmem <= 232448, "split-K GEMM exceeds 227 KB of shared memory");
 
 struct GemmParams {
@@ -56,11 +57,21 @@ struct GemmParams {
   uint32_t* err;
   uint64_t wait_ns;
   // the transform warps scale row r of stage kb by
-  // 2^(pref[kb, r] - rowstat[r].x) * rowstat[r].y (times s_v for FP8)
-  const float* pref;       // [V / 64][R]
+  // 2^(pref[kb, r] - rowstat[r].x) * rowstat[r].y (times s_v for FP8); the
+  // producer copies each stage's 128 references next to the tiles
+  const float* pref;       // [V / 64][R], 16-byte aligned
   const float2* rowstat;   // [R] (m2, 1 / S)
   const float* e_scale;    // FP8 embedder: per-vocabulary-row scales folded into P, else null
 };
+
+// Untiled bulk copy of `bytes` (a multiple of 16; both addresses 16-byte
+// aligned) from global memory into this CTA's shared memory, completing on
+// this CTA's barrier `bar`.
+DG_DEV void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+               : "memory");
+}
 
 // Unit u: d tile n (fastest, so pairs running at once share the P slice in
 // L2), row tile m, K slice q covering stages [k0, k1).
@@ -84,7 +95,8 @@ selfcond_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + kGemmStages * kTileBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + kGemmStages * kTileBytes);
+  float* sRef = reinterpret_cast<float*>(sB + kGemmStages * kTileBytes);  // [stage][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + kGemmStages * (kTileBytes + kRefBytes));
   // barriers: full[S], empty[S], tfull[2], tempty[2], ready[S]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * kGemmStages + 4);
 
@@ -138,15 +150,18 @@ selfcond_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             ok = false;
             break;
           }
-          // this CTA's transform warps wait for its own tiles
+          // this CTA's transform warps wait for its own tiles and the
+          // stage's block references (512 contiguous bytes of [V / 64][R])
           const uint32_t fb = full_bar(stage);
-          mbar_arrive_expect_tx(fb, 2 * kTileBytes);
+          mbar_arrive_expect_tx(fb, 2 * kTileBytes + kRefBytes);
           const uint32_t fb_dst = mapa_shared(fb, rank);
           const int kx = kb * kBlockK;
-          tma_load_2d_pair(smem_u32(sA + stage * kTileBytes), &tmA, fb_dst, kx,
-                           m * kPairM + static_cast<int>(rank) * kBlockM, pol);
+          const int row0 = m * kPairM + static_cast<int>(rank) * kBlockM;
+          tma_load_2d_pair(smem_u32(sA + stage * kTileBytes), &tmA, fb_dst, kx, row0, pol);
           tma_load_2d_pair(smem_u32(sB + stage * kTileBytes), &tmB, fb_dst, kx,
                            n * kBlockN + static_cast<int>(rank) * kHalfN, pol);
+          bulk_load_1d(smem_u32(sRef + stage * kBlockM), p.pref + static_cast<size_t>(kb) * p.R + row0, kRefBytes,
+                       fb);
           if (++stage == kGemmStages) {
             stage = 0;
             phase ^= 1u;
@@ -225,13 +240,12 @@ selfcond_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         const int row = m * kPairM + static_cast<int>(rank) * kBlockM + t;
         const float2 st = __ldg(p.rowstat + row);
         for (int kb = k0; kb < k1; ++kb) {
-          const float ref = __ldg(p.pref + static_cast<size_t>(kb) * p.R + row);
-          const float f = exp2f(ref - st.x) * st.y;
           if (ok && !mbar_wait_bounded(full_bar(stage), phase, p.wait_ns)) {
             atomicOr(p.err, kErrWaitEpilogue);
             ok = false;
           }
           if (ok) {
+            const float f = exp2f(sRef[stage * kBlockM + t] - st.x) * st.y;
             uint4* rp = reinterpret_cast<uint4*>(sA + stage * kTileBytes + t * 128);
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
