@@ -309,7 +309,6 @@ def loop_report(dg, E, E_bits, e_scale, fp8, ws_dtype, torch, B=1):
         # steps' stand-in states in both, so only the loop mechanics differ.
         table = torch.stack([torch.from_numpy(synth.loop_hidden(k, y, E_bits, seed=4).view(np.int16))
                              .view(torch.bfloat16).reshape(-1) for k in range(48)]).cuda()
-        p48 = dg.Params(stop_entropy=0.0)
 
         def fresh():
             canvas.copy_(torch.from_numpy(synth.canvas_uniform(B, L, V, seed=0)))
@@ -323,23 +322,31 @@ def loop_report(dg, E, E_bits, e_scale, fp8, ws_dtype, torch, B=1):
         with torch.cuda.graph(g):
             idx = state.k.to(torch.int64).clamp(0, 47)
             h_buf.view(-1).copy_(torch.index_select(table, 0, idx)[0])
-        out = {}
-        for name in ("host", "device", "host2", "device2"):
-            hp48 = fresh()
+
+        def run(kind, n_steps):
+            p_n = dg.Params(stop_entropy=0.0, max_steps=n_steps)
+            hp_n = fresh()
             torch.cuda.synchronize()
             t0 = time.perf_counter()
-            if name.startswith("host"):
-                n = dg.denoise_loop(E, host_hidden, h_buf, canvas, prev, hp48, acc, ent, samp, amax, stop, ws,
-                                    p48, e_scale=e_scale)
+            if kind == "host":
+                dg.denoise_loop(E, host_hidden, h_buf, canvas, prev, hp_n, acc, ent, samp, amax, stop, ws, p_n,
+                                e_scale=e_scale)
             else:
-                n = dg.denoise_loop_graph(E, g, h_buf, canvas, prev, hp48, acc, ent, samp, amax, stop, ws, state,
-                                          p48, e_scale=e_scale)
+                dg.denoise_loop_graph(E, g, h_buf, canvas, prev, hp_n, acc, ent, samp, amax, stop, ws, state, p_n,
+                                      e_scale=e_scale)
             torch.cuda.synchronize()
-            out[name] = (time.perf_counter() - t0) * 1e6 / int(n[0])
-        timing = {"steps": 48, "host_loop_us_per_step": min(out["host"], out["host2"]),
-                  "device_loop_us_per_step": min(out["device"], out["device2"]),
-                  "what": "wall time of one whole 48-step loop call / 48 (the device loop's includes building and "
-                          "instantiating its graph); stopping disabled, hidden states from a device table"}
+            return (time.perf_counter() - t0) * 1e6
+
+        timing = {"what": "wall time of whole loop calls with stopping disabled (stop entropy 0), hidden states "
+                          "copied from a device table of the stand-in states; per step = slope between 48- and "
+                          "16-step calls, per call = the rest (the device loop builds and instantiates its graph "
+                          "in every call)"}
+        for kind in ("host", "device"):
+            t48 = min(run(kind, 48) for _ in range(2))
+            t16 = min(run(kind, 16) for _ in range(2))
+            slope = (t48 - t16) / 32.0
+            timing[kind + "_loop_us_per_step"] = slope
+            timing[kind + "_loop_us_per_call"] = t16 - 16.0 * slope
         del table, g
     rep = {"steps_at_stop": int(steps.max()) if B == 1 else [int(v) for v in np.bincount(steps)],
             "steps_at_stop_is": "steps run" if B == 1 else "histogram over canvases of the steps each ran",
@@ -416,12 +423,30 @@ def main():
                         dev["prev"], dev["acc"], dev["ent"], dev["samp"], dev["amax"], dev["stop"], ws,
                         params, e_scale=e_scale)
 
+    def head_pass(K):
+        """K steps with CUDA events recorded around every fused head kernel
+        (an event between the head and the merge keeps the merge from
+        launching early, so this pass is kept apart from the step pass);
+        returns the mean head time in ms."""
+        ev_h = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(K)]
+        for a, b in ev_h:       # torch creates the event handles on first record
+            a.record(stream)
+            b.record(stream)
+        torch.cuda.synchronize()
+        for i in range(K):
+            dg.set_head_events(*ev_h[i])
+            step(i, h)
+        dg.set_head_events(None, None)
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in ev_h) / K
+
     def timed_region(K):
-        """K steps timed end to end with nothing else in the stream (the
-        step-throughput pass), then K steps with CUDA events recorded around
-        every fused head kernel (the kernel-time pass: an event between the
-        head and the merge keeps the merge from launching early, so it is
-        kept out of the first pass)."""
+        """The step-throughput pass: K steps timed end to end with nothing
+        else in the stream, bracketed by a kernel-time pass before and one
+        after it, so the head's time is taken under the same power-capped
+        clocks as the steps (their mean)."""
+        head_before = head_pass(K)
         t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if world > 1:
             dist.barrier()
@@ -434,19 +459,8 @@ def main():
         if world > 1:
             dist.barrier()
         total_ms = t0.elapsed_time(t1)
-        ev_h = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in range(K)]
-        for a, b in ev_h:       # torch creates the event handles on first record
-            a.record(stream)
-            b.record(stream)
-        torch.cuda.synchronize()
-        for i in range(K):
-            dg.set_head_events(*ev_h[i])
-            step(i, h)
-        dg.set_head_events(None, None)
-        torch.cuda.synchronize()
-        head_ms = sum(a.elapsed_time(b) for a, b in ev_h) / K
-        return total_ms, head_ms
+        head_after = head_pass(K)
+        return total_ms, 0.5 * (head_before + head_after)
 
     for i in range(args.warmup):
         step(i, h)
@@ -575,8 +589,8 @@ def main():
         sc_line = {"us_per_step": sc_ms * 1e3, "extra_us_over_step": extra_us,
                    "signal_roofline_us": sc_roof_us, "signal_frac": sc_roof_us / extra_us if extra_us > 0 else None,
                    "what": "step + expected-embedding signal [B*256, d] float32 (P bf16 written by the head, "
-                           "split-K tcgen05 GEMM against E^T normalising each landed tile, fixed-order reduction)",
-                   "gpu_launches_per_step": (3 if fp8 else 2) + 2}
+                           "normalisation, split-K tcgen05 GEMM against E^T, fixed-order reduction)",
+                   "gpu_launches_per_step": (3 if fp8 else 2) + 3}
         del ws_sc, E_t
 
     loop = None
@@ -633,8 +647,9 @@ def main():
                     "how": "h uploaded from pinned host memory every step (the next step's upload overlapping "
                            "this step on a second stream), canvas/accept/entropy/stop read back every step"},
             "gpu_launches": (3 if fp8 else 2) * args.steps,
-            "timing": "ms_per_step from K steps with no events in the stream; roofline.kernel_us from a second "
-                      "pass of K steps with events around each fused head kernel",
+            "timing": "ms_per_step from K steps with no events in the stream; roofline.kernel_us the mean of two "
+                      "passes of K steps with events around each fused head kernel, one just before and one just "
+                      "after the step pass",
         }
         if loop is not None:
             line["loop"] = loop

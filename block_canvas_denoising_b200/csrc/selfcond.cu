@@ -13,17 +13,20 @@
 //   1. the fused head (head_sampler.cu), asked for it, also writes block-
 //      scaled probabilities: Pt[r, v] = bf16(2^(z c2 - ref)) for each block
 //      of 64 vocabulary entries with its own reference ref[r, block] (the
-//      running maximum when the block starts), ref to `pref`;
-//   2. normalise: P[r, v] = bf16(Pt[r, v] 2^(ref - m2_r) / S_r [s_v]), with
-//      the row's final maximum m2_r and normaliser S_r from the merge (and
-//      the FP8 embedder's row scales s_v), inside the GEMM: transform warps
-//      scale each row of a landed P tile in shared memory before the MMA
-//      reads it (one factor per row and 64-entry block, which is exactly one
-//      K stage);
+//      running maximum when the block starts), ref to `pref` ([V / 64][R]);
+//   2. normalise (here): P[r, v] = bf16(Pt[r, v] 2^(ref - m2_r) / S_r) in
+//      place, with the row's final maximum m2_r and normaliser S_r from the
+//      merge (and the FP8 embedder's row scale s_v folded in);
 //   3. split-K GEMM (here, tcgen05 pairs): partial[q] = P[:, K_q] . Et[:, K_q]^T
 //      over vocabulary slices K_q, with Et = E^T [d, V] bf16 made once per
 //      embedder (dg_embedder_transpose), so both operands are K-major;
 //   4. reduce (here): s = sum_q partial[q] in a fixed order.
+// The normalisation stays a pass of its own (one read and one write of P).
+// Folding it into the GEMM -- warps rescaling each landed A tile in shared
+// memory before the MMA reads it -- adds a shared-memory read and write of
+// every tile to the TMA write and the MMA read, which already use the SM's
+// shared-memory bandwidth at the MMA rate; measured, that GEMM ran about
+// three times longer than this pass and the plain GEMM together.
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
@@ -42,11 +45,8 @@ namespace {
 // ---------------------------------------------------------------------------
 constexpr int kGemmStages = 6;
 constexpr int kGemmEpiWarps = 8;                       // 4 lane quarters x 2 column halves
-constexpr int kGemmXfWarps = 4;                        // transform: one P row per thread (128 rows)
-constexpr int kGemmXfWarp0 = 2 + kGemmEpiWarps;
-constexpr int kGemmThreads = (2 + kGemmEpiWarps + kGemmXfWarps) * 32;
-constexpr int kRefBytes = kBlockM * 4;  // a stage's block references of this CTA's 128 rows
-constexpr int kGemmSmem = kGemmStages * (2 * kTileBytes + kRefBytes) + 1024 + 256;
+constexpr int kGemmThreads = (2 + kGemmEpiWarps) * 32;
+constexpr int kGemmSmem = kGemmStages * 2 * kTileBytes + 1024 + 256;
 static_assert(kGemmSmem <= 232448, "split-K GEMM exceeds 227 KB of shared memory");
 
 struct GemmParams {
@@ -56,22 +56,7 @@ struct GemmParams {
   float* part;             // [Sk][R][d]
   uint32_t* err;
   uint64_t wait_ns;
-  // the transform warps scale row r of stage kb by
-  // 2^(pref[kb, r] - rowstat[r].x) * rowstat[r].y (times s_v for FP8); the
-  // producer copies each stage's 128 references next to the tiles
-  const float* pref;       // [V / 64][R], 16-byte aligned
-  const float2* rowstat;   // [R] (m2, 1 / S)
-  const float* e_scale;    // FP8 embedder: per-vocabulary-row scales folded into P, else null
 };
-
-// Untiled bulk copy of `bytes` (a multiple of 16; both addresses 16-byte
-// aligned) from global memory into this CTA's shared memory, completing on
-// this CTA's barrier `bar`.
-DG_DEV void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
-               : "memory");
-}
 
 // Unit u: d tile n (fastest, so pairs running at once share the P slice in
 // L2), row tile m, K slice q covering stages [k0, k1).
@@ -84,10 +69,6 @@ DG_DEV void gemm_unit(const GemmParams& p, int u, int& m, int& n, int& q, int& k
   k1 = static_cast<int>((static_cast<int64_t>(q + 1) * p.KB) / p.Sk);
 }
 
-// P arrives block-scaled (the head's Pt) and the transform warps normalise
-// each landed A tile in shared memory; each CTA's loads complete on its own
-// `full` barrier, and the MMA waits for the stage to be both landed and
-// scaled in both CTAs (`ready`, arrivals of both CTAs' transform warps).
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 selfcond_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ GemmParams p) {
@@ -95,10 +76,8 @@ selfcond_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + kGemmStages * kTileBytes;
-  float* sRef = reinterpret_cast<float*>(sB + kGemmStages * kTileBytes);  // [stage][128]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + kGemmStages * (kTileBytes + kRefBytes));
-  // barriers: full[S], empty[S], tfull[2], tempty[2], ready[S]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * kGemmStages + 4);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + kGemmStages * kTileBytes);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kGemmStages + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -109,7 +88,6 @@ selfcond_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
   auto empty_bar = [&](int s) { return smem_u32(&bars[kGemmStages + s]); };
   auto tfull_bar = [&](int a) { return smem_u32(&bars[2 * kGemmStages + a]); };
   auto tempty_bar = [&](int a) { return smem_u32(&bars[2 * kGemmStages + 2 + a]); };
-  auto ready_bar = [&](int s) { return smem_u32(&bars[2 * kGemmStages + 4 + s]); };
 
   if (threadIdx.x == 0) {
     prefetch_tensormap(&tmA);
@@ -122,7 +100,6 @@ selfcond_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       mbar_init(tfull_bar(a), 1);
       mbar_init(tempty_bar(a), 2 * kGemmEpiWarps);
     }
-    for (int s = 0; s < kGemmStages; ++s) mbar_init(ready_bar(s), 2 * kGemmXfWarps);
     fence_mbarrier_init();
   }
   if (warp == 0) {
@@ -150,18 +127,14 @@ selfcond_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             ok = false;
             break;
           }
-          // this CTA's transform warps wait for its own tiles and the
-          // stage's block references (512 contiguous bytes of [V / 64][R])
           const uint32_t fb = full_bar(stage);
-          mbar_arrive_expect_tx(fb, 2 * kTileBytes + kRefBytes);
-          const uint32_t fb_dst = mapa_shared(fb, rank);
+          if (rank == 0) mbar_arrive_expect_tx(fb, 4 * kTileBytes);
+          const uint32_t fb_leader = mapa_shared(fb, 0);
           const int kx = kb * kBlockK;
-          const int row0 = m * kPairM + static_cast<int>(rank) * kBlockM;
-          tma_load_2d_pair(smem_u32(sA + stage * kTileBytes), &tmA, fb_dst, kx, row0, pol);
-          tma_load_2d_pair(smem_u32(sB + stage * kTileBytes), &tmB, fb_dst, kx,
+          tma_load_2d_pair(smem_u32(sA + stage * kTileBytes), &tmA, fb_leader, kx,
+                           m * kPairM + static_cast<int>(rank) * kBlockM, pol);
+          tma_load_2d_pair(smem_u32(sB + stage * kTileBytes), &tmB, fb_leader, kx,
                            n * kBlockN + static_cast<int>(rank) * kHalfN, pol);
-          bulk_load_1d(smem_u32(sRef + stage * kBlockM), p.pref + static_cast<size_t>(kb) * p.R + row0, kRefBytes,
-                       fb);
           if (++stage == kGemmStages) {
             stage = 0;
             phase ^= 1u;
@@ -203,7 +176,7 @@ selfcond_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBlockN);
         for (int kb = k0; kb < k1; ++kb) {
-          if (!mbar_wait_bounded<true>(ready_bar(stage), phase, p.wait_ns)) {
+          if (!mbar_wait_bounded(full_bar(stage), phase, p.wait_ns)) {
             atomicOr(p.err, kErrWaitMmaFull);
             ok = false;
             break;
@@ -222,71 +195,6 @@ selfcond_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
           }
         }
         if (ok) tc_commit_pair_mc(tfull_bar(acc), 0x3);
-      }
-    }
-  } else if (warp >= kGemmXfWarp0) {
-    // ---- transform: thread t scales row t of this CTA's A tile of each
-    // landed stage; a K stage is one 64-entry probability block, so the row
-    // has one factor (the 128-byte swizzle only permutes 16-byte chunks
-    // within the row)
-    {
-      const int t = threadIdx.x - kGemmXfWarp0 * 32;
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int u = pair; u < p.units; u += npairs) {
-        int m, n, q, k0, k1;
-        gemm_unit(p, u, m, n, q, k0, k1);
-        const int row = m * kPairM + static_cast<int>(rank) * kBlockM + t;
-        const float2 st = __ldg(p.rowstat + row);
-        for (int kb = k0; kb < k1; ++kb) {
-          if (ok && !mbar_wait_bounded(full_bar(stage), phase, p.wait_ns)) {
-            atomicOr(p.err, kErrWaitEpilogue);
-            ok = false;
-          }
-          if (ok) {
-            const float f = exp2f(sRef[stage * kBlockM + t] - st.x) * st.y;
-            uint4* rp = reinterpret_cast<uint4*>(sA + stage * kTileBytes + t * 128);
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              // Logical chunk c (entries 8c .. 8c + 7 of the block) sits at
-              // 16-byte slot c ^ (t % 8) under the 128-byte swizzle; visiting
-              // the row in that order puts the lanes of a warp on different
-              // banks (row by row, the same slot would be one bank group)
-              const int slot = c ^ (t & 7);
-              // FP8 embedder: the row scales s_v of the chunk's 8 entries
-              float sv[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
-              if (p.e_scale != nullptr) {
-                const float4* sp = reinterpret_cast<const float4*>(p.e_scale + kb * kBlockK + c * 8);
-                const float4 s0 = __ldg(sp), s1 = __ldg(sp + 1);
-                sv[0] = s0.x; sv[1] = s0.y; sv[2] = s0.z; sv[3] = s0.w;
-                sv[4] = s1.x; sv[5] = s1.y; sv[6] = s1.z; sv[7] = s1.w;
-              }
-              uint4 w = rp[slot];
-              uint32_t* wp = &w.x;
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const __nv_bfloat162 o = __floats2bfloat162_rn(__uint_as_float(wp[j] << 16) * f * sv[2 * j],
-                                                               __uint_as_float(wp[j] & 0xFFFF0000u) * f * sv[2 * j + 1]);
-                wp[j] = *reinterpret_cast<const uint32_t*>(&o);
-              }
-              rp[slot] = w;
-            }
-            // the tensor core reads the tile through the async proxy
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            __syncwarp();
-            if (lane == 0) {
-              if (rank == 0)
-                mbar_arrive(ready_bar(stage));
-              else
-                mbar_arrive_remote(mapa_shared(ready_bar(stage), 0));
-            }
-          }
-          if (++stage == kGemmStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
       }
     }
   } else {
@@ -361,12 +269,39 @@ bool gemm_setup(int* pairs) {
   return true;
 }
 
-int gemm_pairs_of() {
-  static PerDevice<int> cache;
-  int dev = -1, pairs = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
-  if (!cache.get(dev, [](int* v) { return gemm_setup(v); }, &pairs)) return -1;
-  return pairs;
+// ---------------------------------------------------------------------------
+// normalise the block-scaled probabilities in place
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) selfcond_normalize_kernel(uint4* __restrict__ pt, const float* __restrict__ pref,
+                                                                 const float2* __restrict__ rowstat,
+                                                                 const float* __restrict__ e_scale, int R, int V) {
+  const int v8 = V / 8;
+  const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= static_cast<size_t>(R) * v8) return;
+  const int r = static_cast<int>(i / v8);
+  const int v0 = static_cast<int>(i - static_cast<size_t>(r) * v8) * 8;
+  const float2 st = __ldg(rowstat + r);  // (m2, 1 / S)
+  const float ref = __ldg(pref + static_cast<size_t>(v0 / 64) * R + r);  // pref is [V / 64][R]
+  const float f = exp2f(ref - st.x) * st.y;
+  uint4 w = pt[i];
+  uint32_t* wp = &w.x;
+  float sv[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) sv[j] = 1.0f;
+  if (e_scale != nullptr) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(e_scale + v0));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(e_scale + v0) + 1);
+    sv[0] = a.x; sv[1] = a.y; sv[2] = a.z; sv[3] = a.w;
+    sv[4] = b.x; sv[5] = b.y; sv[6] = b.z; sv[7] = b.w;
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float lo = __uint_as_float(wp[j] << 16) * f * sv[2 * j];
+    const float hi = __uint_as_float(wp[j] & 0xFFFF0000u) * f * sv[2 * j + 1];
+    const __nv_bfloat162 o = __floats2bfloat162_rn(lo, hi);
+    wp[j] = *reinterpret_cast<const uint32_t*>(&o);
+  }
+  pt[i] = w;
 }
 
 // ---------------------------------------------------------------------------
@@ -434,7 +369,13 @@ bool encode_kmajor(CUtensorMap* map, const void* base, uint64_t inner, uint64_t 
 
 }  // namespace
 
-int selfcond_gemm_pairs() { return gemm_pairs_of(); }
+int selfcond_gemm_pairs() {
+  static PerDevice<int> cache;
+  int dev = -1, pairs = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (!cache.get(dev, [](int* v) { return gemm_setup(v); }, &pairs)) return -1;
+  return pairs;
+}
 
 int selfcond_slices(int R, int d, int V, int pairs) {
   const int MT = R / kPairM, NT = (d + kBlockN - 1) / kBlockN, KB = V / kBlockK;
@@ -449,8 +390,13 @@ cudaError_t launch_selfcond(const uint16_t* P, const uint16_t* Et, const float* 
                             cudaStream_t stream) {
   const int pairs = selfcond_gemm_pairs();
   if (pairs < 1) return cudaErrorInvalidConfiguration;
-  cudaError_t e;
-  // 2 + 3. normalisation inside the split-K GEMM
+  // 2. normalise
+  const size_t n8 = static_cast<size_t>(R) * (V / 8);
+  selfcond_normalize_kernel<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, stream>>>(
+      reinterpret_cast<uint4*>(const_cast<uint16_t*>(P)), pref, rowstat, e_scale, R, V);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // 3. split-K GEMM
   CUtensorMap tmA, tmB;
   if (!encode_kmajor(&tmA, P, V, R, kBlockM) || !encode_kmajor(&tmB, Et, V, d, kHalfN))
     return cudaErrorInvalidValue;
@@ -467,11 +413,8 @@ cudaError_t launch_selfcond(const uint16_t* P, const uint16_t* Et, const float* 
   gp.part = part;
   gp.err = err;
   gp.wait_ns = kDefaultWaitNs;
-  gp.pref = pref;
-  gp.rowstat = rowstat;
-  gp.e_scale = e_scale;
-  const int use = gp.units < pairs ? gp.units : pairs;
-  selfcond_gemm_kernel<<<2 * use, kGemmThreads, kGemmSmem, stream>>>(tmA, tmB, gp);
+  const int grid = 2 * (gp.units < pairs ? gp.units : pairs);
+  selfcond_gemm_kernel<<<grid, kGemmThreads, kGemmSmem, stream>>>(tmA, tmB, gp);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // 4. reduce
   const size_t n4 = static_cast<size_t>(R) * d / 4;

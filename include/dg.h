@@ -228,8 +228,8 @@ dg_status dg_denoise_loop(const dg_shape* shape, const dg_params* params,
  * trained weights and is out of scope.
  *
  * The head writes block-scaled bf16 probabilities while it samples; a
- * split-K tcgen05 GEMM against E^T (both operands K-major) normalises each
- * landed tile with the merged softmax statistics before multiplying, and a
+ * pass normalises them with the merged softmax statistics, a split-K
+ * tcgen05 GEMM against E^T (both operands K-major) multiplies, and a
  * fixed-order reduction forms s.  P is rounded to bf16 twice (block-scaled, then normalised):
  * |s_gpu - s| <= 2^-8 sum_v p_v |E[v]| per element, plus float32 sums. */
 
