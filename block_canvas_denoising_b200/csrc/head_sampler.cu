@@ -182,15 +182,75 @@ DG_DEV void philox_words8(uint32_t cb, const PhiloxRow& pr, const uint32_t (&rk0
 // wm_pre: when have_wm (warp-uniform), the group's largest Philox word,
 // computed beforehand by another warp; the words themselves are then drawn
 // here only if the group passes its bound.
+// Largest of three floats (finite inputs: the same value as two fmaxf).
+DG_DEV float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Largest of a group's eight Philox words.
+DG_DEV uint32_t max_word8(const uint32_t (&w)[8]) {
+  return __vimax3_u32(__vimax3_u32(w[0], w[1], w[2]), __vimax3_u32(w[3], w[4], w[5]), max(w[6], w[7]));
+}
+
+// Two float32 lanes in one 64-bit register for the packed f32x2 arithmetic
+// (each lane rounds exactly as the scalar instruction).
+DG_DEV uint64_t pack2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+DG_DEV void unpack2(uint64_t v, float& a, float& b) { asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v)); }
+DG_DEV uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+DG_DEV uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// Online softmax partial of a group, base 2: every element below the running
+// maximum adds e = 2^(z c2 - m2) to Sp and (z c2 - m2) e to T2, in two lanes
+// (even and odd elements) folded at the end.  kSel: the group holds the
+// running maximum, whose unit elements are left out; otherwise every element
+// is below it and no test is needed.
+template <bool kSel>
+DG_DEV void softmax8(const float (&z)[8], float c2, Partial& pt) {
+  const float nm = -pt.m2;
+  const uint64_t c22 = pack2(c2, c2), nm2 = pack2(nm, nm);
+  uint64_t s = pack2(0.f, 0.f), t = pack2(0.f, 0.f);
+#pragma unroll
+  for (int j = 0; j < 8; j += 2) {
+    const uint64_t dd = fma2(pack2(z[j], z[j + 1]), c22, nm2);
+    float d0, d1;
+    unpack2(dd, d0, d1);
+    float e0 = ex2_approx(d0), e1 = ex2_approx(d1);
+    if (kSel) {
+      e0 = z[j] < pt.zmax ? e0 : 0.f;
+      e1 = z[j + 1] < pt.zmax ? e1 : 0.f;
+    }
+    const uint64_t ee = pack2(e0, e1);
+    s = add2(s, ee);
+    t = fma2(dd, ee, t);
+  }
+  float s0, s1, t0, t1;
+  unpack2(s, s0, s1);
+  unpack2(t, t0, t1);
+  pt.Sp += s0 + s1;
+  pt.T2 += t0 + t1;
+}
+
 template <bool kHoist>
 DG_DEV void process8(const float (&z)[8], int v0, float inv_tau, float c2, const PhiloxRow& pr,
                      const uint32_t (&rk0)[10], const uint32_t (&rk1)[10], float thr, bool have_wm,
                      uint32_t wm_pre, Partial& pt, Screen& sc) {
   // ---- group max; does the group hold the row's running maximum?  (c2 > 0,
   // so the maximum of z is the maximum of x; groups arrive in increasing v)
-  const float m01 = fmaxf(z[0], z[1]), m23 = fmaxf(z[2], z[3]);
-  const float m45 = fmaxf(z[4], z[5]), m67 = fmaxf(z[6], z[7]);
-  const float gmax = fmaxf(fmaxf(m01, m23), fmaxf(m45, m67));
+  const float gmax = fmax3(fmax3(z[0], z[1], z[2]), fmax3(z[3], z[4], z[5]), fmaxf(z[6], z[7]));
   if (gmax >= pt.zmax) {
     // elements equal to the maximum are units (exponent exactly 0): count
     // them, and find the first (the argmax, ties to the lower index)
@@ -217,28 +277,9 @@ DG_DEV void process8(const float (&z)[8], int v0, float inv_tau, float c2, const
     } else {
       pt.Sp += neq;  // exact ties with the running maximum: more units
     }
-  }
-
-  // ---- online softmax partial, base 2: every element below the maximum
-  {
-    const float nm = -pt.m2;
-    const float zm = pt.zmax;
-    float s0 = 0.f, s1 = 0.f, t0 = 0.f, t1 = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; j += 2) {
-      const float d0 = fmaf(z[j], c2, nm);
-      const float d1 = fmaf(z[j + 1], c2, nm);
-      const float x0 = ex2_approx(d0);
-      const float x1 = ex2_approx(d1);
-      const float e0 = z[j] < zm ? x0 : 0.f;
-      const float e1 = z[j + 1] < zm ? x1 : 0.f;
-      s0 += e0;
-      s1 += e1;
-      t0 = fmaf(d0, e0, t0);
-      t1 = fmaf(d1, e1, t1);
-    }
-    pt.Sp += s0 + s1;
-    pt.T2 += t0 + t1;
+    softmax8<true>(z, c2, pt);
+  } else {
+    softmax8<false>(z, c2, pt);
   }
 
   // ---- Gumbel-max screen (branch-free except for rare near-ties)
@@ -259,7 +300,7 @@ DG_DEV void process8(const float (&z)[8], int v0, float inv_tau, float c2, const
     philox_words8<kHoist>(cb, pr, rk0, rk1, w);
   } else {
     philox_words8<kHoist>(cb, pr, rk0, rk1, w);
-    const uint32_t wm = max(max(max(w[0], w[1]), max(w[2], w[3])), max(max(w[4], w[5]), max(w[6], w[7])));
+    const uint32_t wm = max_word8(w);
     if (__fmaf_rn(lg2_exp1_approx(wm), -kLn2, x0max) < lim_eps) return;
   }
   float kp[8];
@@ -593,7 +634,7 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                                                  static_cast<uint32_t>(canvas_param<kDev>(p, hb).k),
                                                  static_cast<uint32_t>(hb), p.rk0, p.rk1);
         philox_words8<!kFp8>(static_cast<uint32_t>(p.v_off + n_t * kBlockN + g * 8) >> 2, pr, p.rk0, p.rk1, w);
-        dst[g * 32 + r] = max(max(max(w[0], w[1]), max(w[2], w[3])), max(max(w[4], w[5]), max(w[6], w[7])));
+        dst[g * 32 + r] = max_word8(w);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(wfull_bar(buf));
