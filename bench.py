@@ -609,7 +609,18 @@ def main():
         t_tc = flops / (pk["bf16_tflops"] * 1e12)
         gbs = alg_bytes / (head_ms / 1e3) / 1e9
         tflops = flops / (head_ms / 1e3) / 1e12
-        if t_tc > 1.2 * t_hbm:     # the batched step: a dense contraction bound by the tensor cores
+        if t_tc > 1.2 * t_hbm and fp8:
+            # the contraction's own dtype: the E4M3 MMAs issued (two per K
+            # step, 4 R D V flops) against the E4M3 peak, taken as the
+            # measured bf16 peak x 2 (the nominal fp8 / bf16 ratio)
+            roof = {"bound": "tensor", "achieved": 2.0 * tflops, "peak": 2.0 * pk["bf16_tflops"],
+                    "unit": "TFLOP/s", "frac": tflops / pk["bf16_tflops"], "traffic": traffic,
+                    "peak_kind": f"{pk_kind} burst bf16 GEMM x 2 (nominal e4m3 / bf16 ratio)",
+                    "flops_counted": "E4M3 MMA flops issued: two MMAs (h1, h2) per K step, 4 R d V",
+                    "frac_of_sustained": tflops / pk["bf16_tflops_sustained"],
+                    "sustained_peak": 2.0 * pk["bf16_tflops_sustained"],
+                    "hbm_gbs": gbs}
+        elif t_tc > 1.2 * t_hbm:   # the batched step: a dense contraction bound by the tensor cores
             roof = {"bound": "tensor", "achieved": tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                     "frac": tflops / pk["bf16_tflops"], "traffic": traffic,
                     "peak_kind": f"{pk_kind} (burst bf16 GEMM)",

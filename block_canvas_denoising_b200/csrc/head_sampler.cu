@@ -120,10 +120,17 @@ struct Screen {
   float z1;        // its logit
   uint32_t w1;     // its Philox word
   int v1;          // its vocabulary index
+  float lim_eps;   // the group bound's limit: max(K1a, thr) less its margin
 };
 
 DG_DEV float screen_eps(float k) {
   return 2.0f * kGumbelApproxErr + (fabsf(k) + 64.0f) * 1.9073486328125e-06f;  // 2^-19
+}
+
+// The group bound's limit, formed when thr (per tile) or K1a changes.
+DG_DEV void screen_limit(Screen& sc, float thr) {
+  const float lim = fmaxf(sc.K1a, thr);
+  sc.lim_eps = lim - 2.0f * screen_eps(lim);
 }
 
 DG_DEV void screen_reset(Screen& sc) { sc.K1a = -FLT_MAX; }
@@ -289,8 +296,7 @@ DG_DEV void process8(const float (&z)[8], int v0, float inv_tau, float c2, const
   // row, no element of the group can win or tie: skip it (first with the
   // largest possible noise, before any Philox work, then with the group's).
   // The margin covers the screen's error on both keys and the index packing.
-  const float lim = fmaxf(sc.K1a, thr);
-  const float lim_eps = lim - 2.0f * screen_eps(lim);
+  const float lim_eps = sc.lim_eps;
   const float x0max = __fmaf_rn(gmax, inv_tau, kGumbelC0);
   if (x0max + (kGumbelMaxNoise + 1e-3f - kGumbelC0) < lim_eps) return;
   const uint32_t cb = static_cast<uint32_t>(v0) >> 2;
@@ -338,6 +344,7 @@ DG_DEV void process8(const float (&z)[8], int v0, float inv_tau, float c2, const
     sc.z1 = zs;
     sc.w1 = ws;
     sc.v1 = v0 + j1;
+    screen_limit(sc, thr);
   }
 }
 
@@ -712,6 +719,7 @@ head_sampler_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         const float thr = fmaxf(fmaxf(fmaxf(sRec[0 * kBlockM + rloc], sRec[1 * kBlockM + rloc]),
                                       fmaxf(sRec[2 * kBlockM + rloc], sRec[3 * kBlockM + rloc])),
                                 key_order_dec(grec));
+        screen_limit(sc, thr);
         grec = __ldcg(p.row_rec + row);
         uint32_t ra[8], rb[8];
         float blk_ref = 0.f;  // self-conditioning: this tile's 64-entry block reference
