@@ -323,6 +323,10 @@ def loop_report(dg, E, E_bits, e_scale, fp8, ws_dtype, torch, B=1):
             idx = state.k.to(torch.int64).clamp(0, 47)
             h_buf.view(-1).copy_(torch.index_select(table, 0, idx)[0])
 
+        # the device loop built once per schedule length and run again
+        handles = {n: dg.LoopGraph(E, g, h_buf, canvas, prev, acc, ent, samp, amax, stop, ws, state,
+                                   dg.Params(stop_entropy=0.0, max_steps=n), e_scale=e_scale) for n in (16, 48)}
+
         def run(kind, n_steps):
             p_n = dg.Params(stop_entropy=0.0, max_steps=n_steps)
             hp_n = fresh()
@@ -331,22 +335,27 @@ def loop_report(dg, E, E_bits, e_scale, fp8, ws_dtype, torch, B=1):
             if kind == "host":
                 dg.denoise_loop(E, host_hidden, h_buf, canvas, prev, hp_n, acc, ent, samp, amax, stop, ws, p_n,
                                 e_scale=e_scale)
-            else:
+            elif kind == "device":
                 dg.denoise_loop_graph(E, g, h_buf, canvas, prev, hp_n, acc, ent, samp, amax, stop, ws, state, p_n,
                                       e_scale=e_scale)
+            else:
+                handles[n_steps].run(hp_n)
             torch.cuda.synchronize()
             return (time.perf_counter() - t0) * 1e6
 
         timing = {"what": "wall time of whole loop calls with stopping disabled (stop entropy 0), hidden states "
                           "copied from a device table of the stand-in states; per step = slope between 48- and "
-                          "16-step calls, per call = the rest (the device loop builds and instantiates its graph "
-                          "in every call)"}
-        for kind in ("host", "device"):
+                          "16-step calls, per call = the rest (device: dg_denoise_loop_graph, which builds and "
+                          "instantiates its graph in every call; device_built: a dg_loop_graph handle built once "
+                          "and run again)"}
+        for kind in ("host", "device", "device_built"):
             t48 = min(run(kind, 48) for _ in range(2))
             t16 = min(run(kind, 16) for _ in range(2))
             slope = (t48 - t16) / 32.0
             timing[kind + "_loop_us_per_step"] = slope
             timing[kind + "_loop_us_per_call"] = t16 - 16.0 * slope
+        for hdl in handles.values():
+            hdl.close()
         del table, g
     rep = {"steps_at_stop": int(steps.max()) if B == 1 else [int(v) for v in np.bincount(steps)],
             "steps_at_stop_is": "steps run" if B == 1 else "histogram over canvases of the steps each ran",
@@ -401,13 +410,20 @@ def main():
         e_scale = None
     h = torch.from_numpy(h_bits.view(np.int16)).view(torch.bfloat16).cuda()
     R = B * L
-    dev = dict(canvas=torch.zeros(R, dtype=torch.int32, device="cuda"),
+    # the four results read back every step (canvas, accept, entropy, stop)
+    # live in one device buffer, so the end-to-end pass reads them with one
+    # copy per step
+    off_acc, off_ent = 4 * R, 4 * R + ((R + 15) // 16) * 16
+    off_stop = off_ent + 4 * R
+    res_bytes = off_stop + 4 * B
+    res_dev = torch.zeros(res_bytes, dtype=torch.uint8, device="cuda")
+    dev = dict(canvas=res_dev[:off_acc].view(torch.int32),
                prev=torch.zeros(R, dtype=torch.int32, device="cuda"),
-               acc=torch.zeros(R, dtype=torch.uint8, device="cuda"),
-               ent=torch.zeros(R, dtype=torch.float32, device="cuda"),
+               acc=res_dev[off_acc:off_acc + R],
+               ent=res_dev[off_ent:off_stop].view(torch.float32),
                samp=torch.zeros(R, dtype=torch.int32, device="cuda"),
                amax=torch.zeros(R, dtype=torch.int32, device="cuda"),
-               stop=torch.zeros(B, dtype=torch.int32, device="cuda"))
+               stop=res_dev[off_stop:].view(torch.int32))
     ws_dtype = dg.E_FP8_E4M3 if fp8 else dg.E_BF16
     ws = dg.Workspace(B, D, V, ws_dtype)
     params = dg.Params(seed=philox_seed)
@@ -508,10 +524,9 @@ def main():
     # step's stream.
     h_host = torch.from_numpy(h_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
     h_dev = [torch.empty_like(h), torch.empty_like(h)]
-    outs = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory()
-            for k, v in dev.items() if k in ("canvas", "acc", "ent", "stop")}
+    res_host = torch.empty(res_bytes, dtype=torch.uint8).pin_memory()
     h2d = h_host.numel() * 2
-    d2h = sum(o.numel() * o.element_size() for o in outs.values())
+    d2h = res_bytes
     K2 = max(1, args.steps)
     up = torch.cuda.Stream()
     ready = [torch.cuda.Event(), torch.cuda.Event()]
@@ -540,10 +555,7 @@ def main():
         stream.wait_event(ready[j])
         step(i, h_dev[j])
         consumed[j].record(stream)
-        outs["canvas"].copy_(dev["canvas"], non_blocking=True)
-        outs["acc"].copy_(dev["acc"], non_blocking=True)
-        outs["ent"].copy_(dev["ent"], non_blocking=True)
-        outs["stop"].copy_(dev["stop"], non_blocking=True)
+        res_host.copy_(res_dev, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
     (e2e_total,) = reduce_max([e0.elapsed_time(e1)], dist, "cuda")
@@ -656,7 +668,8 @@ def main():
             "e2e": {"value": e2e_value, "unit": "slots/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                     "how": "h uploaded from pinned host memory every step (the next step's upload overlapping "
-                           "this step on a second stream), canvas/accept/entropy/stop read back every step"},
+                           "this step on a second stream), canvas/accept/entropy/stop read back every step in one copy "
+                           "(the four outputs share one device buffer)"},
             "gpu_launches": (3 if fp8 else 2) * args.steps,
             "timing": "ms_per_step from K steps with no events in the stream; roofline.kernel_us the mean of two "
                       "passes of K steps with events around each fused head kernel, one just before and one just "

@@ -129,6 +129,14 @@ def lib() -> ctypes.CDLL:
                                             ctypes.c_int32, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P,
                                             ctypes.c_size_t, P]
         L.dg_denoise_loop_graph.restype = ctypes.c_int
+        L.dg_loop_graph_create.argtypes = [ctypes.POINTER(_Shape), ctypes.POINTER(_Params), P, P, P, P, P, P,
+                                           P, P, P, P, P, P, ctypes.c_size_t, P, ctypes.c_size_t,
+                                           ctypes.POINTER(ctypes.c_void_p)]
+        L.dg_loop_graph_create.restype = ctypes.c_int
+        L.dg_loop_graph_run.argtypes = [P, ctypes.c_int32, P, P, P]
+        L.dg_loop_graph_run.restype = ctypes.c_int
+        L.dg_loop_graph_destroy.argtypes = [P]
+        L.dg_loop_graph_destroy.restype = None
         L.dg_init_canvas.argtypes = [ctypes.POINTER(_Shape), ctypes.POINTER(_Params), P, P]
         L.dg_init_canvas.restype = ctypes.c_int
         L.dg_generate_blocks.argtypes = [ctypes.POINTER(_Shape), ctypes.POINTER(_Params), P, P, ctypes.c_int32,
@@ -374,6 +382,53 @@ def denoise_loop_graph(E, hidden_graph, h_buf, canvas, prev_argmax, has_prev, ac
         _ptr(stop), _ptr(state.buf), ctypes.c_size_t(state.nbytes), _ptr(ws.buf), ctypes.c_size_t(ws.nbytes),
         _stream(stream)), "dg_denoise_loop_graph")
     return steps
+
+
+class LoopGraph:
+    """The device-side loop built once and run many times
+    (``dg_loop_graph_create`` / ``_run`` / ``_destroy``): the buffers are
+    fixed at construction (they must outlive the object); ``run`` takes the
+    first step, the host uint8 ``has_prev`` array (updated in place) and
+    returns the host int32 array of steps taken."""
+
+    def __init__(self, E, hidden_graph, h_buf, canvas, prev_argmax, accept, entropy, sampled, argmax, stop,
+                 ws: Workspace, state: LoopState, params: Params = Params(), e_scale=None):
+        B = int(stop.shape[0])
+        R, d = h_buf.shape
+        V = E.shape[0]
+        e_dtype = E_BF16 if e_scale is None else E_FP8_E4M3
+        self.B = B
+        shp = _shape(B, d, V, e_dtype, L=R // B)
+        prm = params.c()
+        g = None if hidden_graph is None else ctypes.c_void_p(int(hidden_graph.raw_cuda_graph()))
+        handle = ctypes.c_void_p()
+        # the buffers stay referenced for the handle's lifetime
+        self._keep = (E, e_scale, h_buf, canvas, prev_argmax, accept, entropy, sampled, argmax, stop, ws, state)
+        self._h = None
+        _check(lib().dg_loop_graph_create(
+            ctypes.byref(shp), ctypes.byref(prm), _ptr(E), _ptr(e_scale), g, _ptr(h_buf), _ptr(canvas),
+            _ptr(prev_argmax), _ptr(accept), _ptr(entropy), _ptr(sampled), _ptr(argmax), _ptr(stop),
+            _ptr(state.buf), ctypes.c_size_t(state.nbytes), _ptr(ws.buf), ctypes.c_size_t(ws.nbytes),
+            ctypes.byref(handle)), "dg_loop_graph_create")
+        self._h = handle
+
+    def run(self, has_prev, k_start: int = 0, stream=None):
+        assert isinstance(has_prev, np.ndarray) and has_prev.dtype == np.uint8 and len(has_prev) == self.B
+        steps = np.zeros(self.B, np.int32)
+        _check(lib().dg_loop_graph_run(self._h, ctypes.c_int32(k_start), has_prev.ctypes.data_as(ctypes.c_void_p),
+                                       steps.ctypes.data_as(ctypes.c_void_p), _stream(stream)), "dg_loop_graph_run")
+        return steps
+
+    def close(self) -> None:
+        if self._h is not None:
+            lib().dg_loop_graph_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def embedder_transpose(E, E_t, e_fp8: bool = False, stream=None) -> None:

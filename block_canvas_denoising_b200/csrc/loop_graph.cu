@@ -11,17 +11,22 @@
 // advance k, prepare the next step's per-canvas data (step word, 1/tau in
 // float64 exactly as the host computes it) and the list of canvases still
 // running -- then sets the while condition.  Nothing returns to the host
-// until every canvas is done.
+// until every canvas is done.  The graph holds no per-call value, so it can
+// be built once (dg_loop_graph_create) and run many times
+// (dg_loop_graph_run): an init kernel writes the call's first step and
+// previous-prediction flags into the loop state before each launch.
 //
 // Loop state (caller-owned device memory, dg_loop_state_bytes(B) bytes):
 //   offset 0   int32 k, the step the body is about to run (the hidden-state
 //              graph reads it), then int32 canvases still running, int32
-//              steps run, int32 stop reason (0 running, 1 done, 2 fault)
+//              steps run, int32 stop reason (0 running, 1 done, 2 fault),
+//              int32 the call's first step
 //   offset 256 CanvasParam[B], then uint8 canvas_of[B], uint8 has_prev[B],
 //              uint8 active[B] (256-byte aligned each), int32 steps[B].
 #include <string.h>
 
 #include <mutex>
+#include <new>
 
 #include "dg_device.cuh"
 #include "dg_internal.h"
@@ -53,9 +58,13 @@ struct LoopHeader {
   int32_t n_active;
   int32_t iterations;
   int32_t reason;
+  int32_t k_start;  // the call's first step (the graph itself holds no per-call value)
 };
 
-// Everything the init and control kernels need; passed by value.
+// Everything the init and control kernels need; passed by value.  The
+// control kernel is captured into the graph, so it reads the per-call
+// values (k_start, has_prev) from the loop state, which the init kernel
+// writes before each launch.
 struct LoopCtl {
   LoopHeader* hdr;
   CanvasParam* cp;
@@ -118,6 +127,7 @@ __global__ void __launch_bounds__(256) loop_init_kernel(const __grid_constant__ 
   }
   if (b == 0) {
     c.hdr->k = c.k_start;
+    c.hdr->k_start = c.k_start;
     c.hdr->iterations = 0;
     c.hdr->reason = 0;
   }
@@ -127,8 +137,11 @@ __global__ void __launch_bounds__(256) loop_init_kernel(const __grid_constant__ 
 
 __global__ void __launch_bounds__(256) loop_control_kernel(const __grid_constant__ LoopCtl c) {
   __shared__ uint8_t s_commit[DG_MAX_B];
-  __shared__ int s_k;
-  if (threadIdx.x == 0) s_k = c.hdr->k;
+  __shared__ int s_k, s_k0;
+  if (threadIdx.x == 0) {
+    s_k = c.hdr->k;
+    s_k0 = c.hdr->k_start;
+  }
   __syncthreads();
   const int k = s_k;
   const int b = threadIdx.x;
@@ -141,7 +154,7 @@ __global__ void __launch_bounds__(256) loop_control_kernel(const __grid_constant
         // tokens and is frozen
         commit = 1;
         c.active[b] = 0;
-        c.steps[b] = k - c.k_start + 1;
+        c.steps[b] = k - s_k0 + 1;
       }
     }
     s_commit[b] = commit;
@@ -191,19 +204,28 @@ extern "C" size_t dg_loop_state_bytes(int32_t B) {
   return loop_layout(B).total;
 }
 
-extern "C" dg_status dg_denoise_loop_graph(const dg_shape* shape, const dg_params* params, const void* E,
-                                           const float* e_scale, void* hidden_graph, int32_t k_start,
-                                           void* h_buf, int32_t* canvas, int32_t* prev_argmax, uint8_t* has_prev,
-                                           int32_t* steps_taken, uint8_t* accept, float* entropy,
-                                           int32_t* sampled, int32_t* argmax, int32_t* stop, void* loop_state,
-                                           size_t state_bytes, void* workspace, size_t ws_bytes, void* stream) {
+// The built loop behind a dg_loop_graph handle.
+struct dg_loop_graph_s {
+  LoopCtl c;
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  int device = -1;
+  void* workspace = nullptr;
+  size_t ws_bytes = 0;
+};
+
+extern "C" dg_status dg_loop_graph_create(const dg_shape* shape, const dg_params* params, const void* E,
+                                          const float* e_scale, void* hidden_graph, void* h_buf, int32_t* canvas,
+                                          int32_t* prev_argmax, uint8_t* accept, float* entropy, int32_t* sampled,
+                                          int32_t* argmax, int32_t* stop, void* loop_state, size_t state_bytes,
+                                          void* workspace, size_t ws_bytes, dg_loop_graph* out) {
+  if (out == nullptr) return DG_ERR_INVALID_ARG;
+  *out = nullptr;
   dg_status st = check_shape_and_params(shape, params);
   if (st != DG_OK) return st;
-  if (has_prev == nullptr || steps_taken == nullptr || loop_state == nullptr || h_buf == nullptr ||
-      canvas == nullptr || workspace == nullptr)
+  if (loop_state == nullptr || h_buf == nullptr || canvas == nullptr || workspace == nullptr)
     return DG_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(loop_state) & 255u) != 0) return DG_ERR_INVALID_ARG;
-  if (k_start < 0 || k_start >= params->max_steps) return DG_ERR_RANGE;
   const int B = shape->B;
   const LoopLayout lay = loop_layout(B);
   if (state_bytes < lay.total) return DG_ERR_WORKSPACE;
@@ -211,7 +233,8 @@ extern "C" dg_status dg_denoise_loop_graph(const dg_shape* shape, const dg_param
   const size_t ws_need = dg_workspace_size(shape);
   if (ws_need == 0) return DG_ERR_NO_DEVICE;
   if (ws_bytes < ws_need) return DG_ERR_WORKSPACE;
-  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DG_ERR_NO_DEVICE;
   uint8_t* base = static_cast<uint8_t*>(loop_state);
 
   LoopCtl c;
@@ -229,12 +252,10 @@ extern "C" dg_status dg_denoise_loop_graph(const dg_shape* shape, const dg_param
   c.B = B;
   c.L = shape->L;
   c.N = params->max_steps;
-  c.k_start = k_start;
   c.block = params->block;
   c.tau0 = params->tau0;
   c.tau1 = params->tau1;
-  for (int b = 0; b < B; ++b) c.has_prev_in[b] = has_prev[b] ? 1 : 0;
-  LoopDevState dev{c.cp, c.canvas_of, &c.hdr->n_active};
+  LoopDevState devst{c.cp, c.canvas_of, &c.hdr->n_active};
 
   // ---- the graph: while (condition) { hidden graph; step; control }
   cudaStream_t cap;
@@ -242,7 +263,6 @@ extern "C" dg_status dg_denoise_loop_graph(const dg_shape* shape, const dg_param
   cudaGraph_t graph = nullptr;
   cudaGraphExec_t exec = nullptr;
   cudaGraphConditionalHandle handle;
-  st = DG_OK;
   {
     std::lock_guard<std::mutex> lock(g_capture_mu);
     if (cudaGraphCreate(&graph, 0) != cudaSuccess) return DG_ERR_CUDA;
@@ -278,8 +298,10 @@ extern "C" dg_status dg_denoise_loop_graph(const dg_shape* shape, const dg_param
       set_last_error_message("capture of the loop body failed to start");
       return DG_ERR_CUDA;
     }
-    st = enqueue_loop_step(shape, params, h_buf, E, e_scale, k_start, canvas, prev_argmax, accept, entropy,
-                           sampled, argmax, stop, workspace, ws_bytes, &dev, cap);
+    // the step's kernels read the per-canvas step words from the loop
+    // state; the step index passed here only satisfies the range check
+    st = enqueue_loop_step(shape, params, h_buf, E, e_scale, 0, canvas, prev_argmax, accept, entropy, sampled,
+                           argmax, stop, workspace, ws_bytes, &devst, cap);
     if (st == DG_OK) {
       loop_control_kernel<<<1, 256, 0, cap>>>(c);
       if (cudaGetLastError() != cudaSuccess) st = DG_ERR_CUDA;
@@ -295,25 +317,88 @@ extern "C" dg_status dg_denoise_loop_graph(const dg_shape* shape, const dg_param
       st = DG_ERR_CUDA;
     }
   }
-  if (st == DG_OK) {
-    loop_init_kernel<<<1, 256, 0, cs>>>(c);
-    if (cudaGetLastError() != cudaSuccess || cudaGraphLaunch(exec, cs) != cudaSuccess) st = DG_ERR_CUDA;
+  if (st != DG_OK) {
+    if (exec != nullptr) cudaGraphExecDestroy(exec);
+    cudaGraphDestroy(graph);
+    return st;
+  }
+  dg_loop_graph g = new (std::nothrow) dg_loop_graph_s;
+  if (g == nullptr) {
+    cudaGraphExecDestroy(exec);
+    cudaGraphDestroy(graph);
+    return DG_ERR_CUDA;
+  }
+  g->c = c;
+  g->graph = graph;
+  g->exec = exec;
+  g->device = dev;
+  g->workspace = workspace;
+  g->ws_bytes = ws_bytes;
+  *out = g;
+  return DG_OK;
+}
+
+extern "C" dg_status dg_loop_graph_run(dg_loop_graph g, int32_t k_start, uint8_t* has_prev, int32_t* steps_taken,
+                                       void* stream) {
+  if (g == nullptr || has_prev == nullptr || steps_taken == nullptr) return DG_ERR_INVALID_ARG;
+  if (k_start < 0 || k_start >= g->c.N) return DG_ERR_RANGE;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != g->device) {
+    set_last_error_message("dg_loop_graph_run: the graph was built on another device");
+    return DG_ERR_INVALID_ARG;
+  }
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  LoopCtl c = g->c;
+  c.k_start = k_start;
+  for (int b = 0; b < c.B; ++b) c.has_prev_in[b] = has_prev[b] ? 1 : 0;
+  loop_init_kernel<<<1, 256, 0, cs>>>(c);
+  if (cudaGetLastError() != cudaSuccess || cudaGraphLaunch(g->exec, cs) != cudaSuccess) {
+    set_last_error_message("launching the loop graph failed");
+    return DG_ERR_CUDA;
   }
   int32_t steps_h[DG_MAX_B];
   uint8_t hp_h[DG_MAX_B];
-  if (st == DG_OK &&
-      (cudaMemcpyAsync(steps_h, c.steps, sizeof(int32_t) * B, cudaMemcpyDeviceToHost, cs) != cudaSuccess ||
-       cudaMemcpyAsync(hp_h, c.has_prev, B, cudaMemcpyDeviceToHost, cs) != cudaSuccess ||
-       cudaStreamSynchronize(cs) != cudaSuccess))
-    st = DG_ERR_CUDA;
-  if (exec != nullptr) cudaGraphExecDestroy(exec);
-  if (graph != nullptr) cudaGraphDestroy(graph);
-  if (st != DG_OK) return st;
-  for (int b = 0; b < B; ++b) {
+  if (cudaMemcpyAsync(steps_h, c.steps, sizeof(int32_t) * c.B, cudaMemcpyDeviceToHost, cs) != cudaSuccess ||
+      cudaMemcpyAsync(hp_h, c.has_prev, c.B, cudaMemcpyDeviceToHost, cs) != cudaSuccess ||
+      cudaStreamSynchronize(cs) != cudaSuccess) {
+    set_last_error_message("reading the loop's results failed");
+    return DG_ERR_CUDA;
+  }
+  for (int b = 0; b < c.B; ++b) {
     steps_taken[b] = steps_h[b];
     has_prev[b] = hp_h[b];
   }
   // a bounded wait that ran out (or a non-finite FP8 hidden state) stopped
   // the loop early: report it
-  return dg_device_status(workspace, ws_bytes, stream);
+  return dg_device_status(g->workspace, g->ws_bytes, stream);
+}
+
+extern "C" void dg_loop_graph_destroy(dg_loop_graph g) {
+  if (g == nullptr) return;
+  int cur = -1;
+  const bool switch_dev = cudaGetDevice(&cur) == cudaSuccess && cur != g->device;
+  if (switch_dev) cudaSetDevice(g->device);
+  if (g->exec != nullptr) cudaGraphExecDestroy(g->exec);
+  if (g->graph != nullptr) cudaGraphDestroy(g->graph);
+  if (switch_dev) cudaSetDevice(cur);
+  delete g;
+}
+
+extern "C" dg_status dg_denoise_loop_graph(const dg_shape* shape, const dg_params* params, const void* E,
+                                           const float* e_scale, void* hidden_graph, int32_t k_start,
+                                           void* h_buf, int32_t* canvas, int32_t* prev_argmax, uint8_t* has_prev,
+                                           int32_t* steps_taken, uint8_t* accept, float* entropy,
+                                           int32_t* sampled, int32_t* argmax, int32_t* stop, void* loop_state,
+                                           size_t state_bytes, void* workspace, size_t ws_bytes, void* stream) {
+  dg_status st = check_shape_and_params(shape, params);
+  if (st != DG_OK) return st;
+  if (has_prev == nullptr || steps_taken == nullptr) return DG_ERR_INVALID_ARG;
+  if (k_start < 0 || k_start >= params->max_steps) return DG_ERR_RANGE;
+  dg_loop_graph g = nullptr;
+  st = dg_loop_graph_create(shape, params, E, e_scale, hidden_graph, h_buf, canvas, prev_argmax, accept, entropy,
+                            sampled, argmax, stop, loop_state, state_bytes, workspace, ws_bytes, &g);
+  if (st != DG_OK) return st;
+  st = dg_loop_graph_run(g, k_start, has_prev, steps_taken, stream);
+  dg_loop_graph_destroy(g);
+  return st;
 }

@@ -296,6 +296,39 @@ dg_status dg_denoise_loop_graph(const dg_shape* shape, const dg_params* params,
                                 void* loop_state, size_t state_bytes,
                                 void* workspace, size_t ws_bytes, void* stream);
 
+/* The same loop built once and run many times: dg_denoise_loop_graph
+ * builds (by stream capture), instantiates and destroys its graph in every
+ * call; a dg_loop_graph keeps it.
+ *
+ * dg_loop_graph_create -- build and instantiate the loop graph on the current
+ * device for fixed buffers.  Arguments as for dg_denoise_loop_graph, less
+ * the per-call ones (k_start, has_prev, steps_taken, stream); every buffer
+ * must stay allocated, and hold its role, until the handle is destroyed.
+ * The hidden-state graph is copied into the loop when the handle is built:
+ * later changes to hidden_graph do not reach it.  On success *out holds the
+ * handle; on failure *out is NULL.
+ *
+ * dg_loop_graph_run -- one adaptive loop from step k_start with the given
+ * has_prev (HOST uint8 [B], in/out) and steps_taken (HOST int32 [B], out),
+ * enqueued on `stream` and synchronised, exactly as dg_denoise_loop_graph
+ * (whose results it equals).  The canvas and prev_argmax buffers given at
+ * create time are the loop's input and output.  Must be called on the
+ * device the handle was built on (else DG_ERR_INVALID_ARG); runs of one
+ * handle must not overlap (they share the loop state and workspace).
+ *
+ * dg_loop_graph_destroy -- release the graph (NULL is a no-op). */
+typedef struct dg_loop_graph_s* dg_loop_graph;
+dg_status dg_loop_graph_create(const dg_shape* shape, const dg_params* params,
+                               const void* E, const float* e_scale, void* hidden_graph,
+                               void* h_buf, int32_t* canvas, int32_t* prev_argmax,
+                               uint8_t* accept, float* entropy, int32_t* sampled,
+                               int32_t* argmax, int32_t* stop,
+                               void* loop_state, size_t state_bytes,
+                               void* workspace, size_t ws_bytes, dg_loop_graph* out);
+dg_status dg_loop_graph_run(dg_loop_graph graph, int32_t k_start, uint8_t* has_prev,
+                            int32_t* steps_taken, void* stream);
+void dg_loop_graph_destroy(dg_loop_graph graph);
+
 /* ---- block-by-block generation ([Report] Figure 4: encode & append) ----
  * Generation runs block after block: each block of B canvases starts from
  * uniform noise, the adaptive loop denoises it until it settles, and the

@@ -184,6 +184,31 @@ def test_device_loop_host_checks(libdg):
     assert call(prm=dg.Params(max_steps=0)) == 1
 
 
+def test_loop_graph_handle_host_checks(libdg):
+    # the reusable device loop refuses bad arguments on the host; without a
+    # device it reports DG_ERR_NO_DEVICE and hands back no handle
+    n1 = libdg.dg_loop_state_bytes(1)
+    shp = dg._Shape(1, 256, 512, 4096, 0)
+    fake = ctypes.c_void_p(4096)
+    P = ctypes.c_void_p
+
+    def create(state=fake, nbytes=n1, prm=dg.Params(), out=True):
+        p = prm.c()
+        h = ctypes.c_void_p(1234)
+        rc = libdg.dg_loop_graph_create(ctypes.byref(shp), ctypes.byref(p), fake, None, None, fake, fake, fake,
+                                        fake, fake, fake, fake, fake, state, ctypes.c_size_t(nbytes), fake,
+                                        ctypes.c_size_t(1 << 30), ctypes.byref(h) if out else None)
+        return rc, h.value
+    assert create(out=False)[0] == 1
+    assert create(state=ctypes.c_void_p(4096 + 16)) == (1, None)   # not 256-byte aligned; *out cleared
+    assert create(nbytes=n1 - 1) == (3, None)
+    assert create(prm=dg.Params(max_steps=0)) == (1, None)
+    hp = np.zeros(1, np.uint8)
+    st = np.zeros(1, np.int32)
+    assert libdg.dg_loop_graph_run(None, 0, hp.ctypes.data_as(P), st.ctypes.data_as(P), None) == 1
+    libdg.dg_loop_graph_destroy(None)                                 # a no-op
+
+
 def test_selfcond_host_checks(libdg):
     # E_t and signal are required and 16-byte aligned; the workspace must
     # hold the signal's scratch (refused before any device work)

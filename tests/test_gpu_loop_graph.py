@@ -221,3 +221,50 @@ def test_loop_stops_on_a_latched_fault(device_loop):
     # one step ran (the outputs are written) but no canvas was committed
     assert int(outs["accept"].sum()) >= B
     assert not np.array_equal(canvas.cpu().numpy(), canvas0)   # renoised by the step, not committed
+
+
+def test_loop_graph_handle_runs_again_and_equals_the_one_shot_loop():
+    # one handle (dg_loop_graph_create) run three times with different
+    # starting canvases, first steps and previous-prediction flags; every
+    # run equals the one-shot dg_denoise_loop_graph on the same inputs, bit
+    # for bit.  The buffers are the handle's: each run's inputs are copied in
+    B, d, V = 2, 256, 1024
+    R = B * L
+    E_bits = synth.embedder_normal(V, d, seed=1)
+    E = to_dev_bf16(E_bits)
+    y = synth.loop_targets(L, V, seed=3, B=B)
+    params = dg.Params(max_steps=12)
+    table = _table(E_bits, y, params.max_steps, 0)
+    h_buf = torch.empty((R, d), dtype=torch.bfloat16, device="cuda")
+    canvas = torch.zeros(R, dtype=torch.int32, device="cuda")
+    prev = torch.zeros(R, dtype=torch.int32, device="cuda")
+    outs = _outs(B)
+    ws = dg.Workspace(B, d, V)
+    state = dg.LoopState(B)
+    g = torch.cuda.CUDAGraph(keep_graph=True)
+    with torch.cuda.graph(g):
+        idx = state.k.to(torch.int64).clamp(0, table.shape[0] - 1)
+        h_buf.view(-1).copy_(torch.index_select(table, 0, idx)[0])
+    lg = dg.LoopGraph(E, g, h_buf, canvas, prev, outs["accept"], outs["entropy"], outs["sampled"], outs["argmax"],
+                      outs["stop"], ws, state, params)
+    rng = np.random.default_rng(7)
+    cases = [(0, np.zeros(B, np.uint8), np.zeros(R, np.int32), 0),
+             (3, np.ones(B, np.uint8), rng.integers(0, V, R).astype(np.int32), 1),
+             (0, np.array([1, 0], np.uint8), rng.integers(0, V, R).astype(np.int32), 2)]
+    try:
+        for k_start, hp0, prev0, seed in cases:
+            canvas0 = synth.canvas_uniform(B, L, V, seed=seed)
+            canvas.copy_(torch.from_numpy(canvas0))
+            prev.copy_(torch.from_numpy(prev0))
+            hp = hp0.copy()
+            steps = lg.run(hp, k_start=k_start)
+            torch.cuda.synchronize()
+            got = {k: v.cpu().numpy() for k, v in outs.items()}
+            got.update(canvas=canvas.cpu().numpy(), prev=prev.cpu().numpy(), has_prev=hp, steps=steps)
+            ref_table = _table(E_bits, y, params.max_steps, k_start) if k_start else table
+            ref = _run_graph(E, ref_table, B, d, V, params, k_start=k_start, canvas0=canvas0, prev0=prev0,
+                             has_prev=hp0.copy())
+            _same(got, ref)
+            assert int(state.k.item()) == int(steps.max()) + k_start
+    finally:
+        lg.close()
