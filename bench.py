@@ -647,6 +647,18 @@ def main():
                      "algorithmic_bytes": alg_bytes, "flops": flops,
                      "step_roofline_us": max(t_hbm, t_tc) * 1e6,
                      "step_frac": max(t_hbm, t_tc) * 1e3 / ms_per_step})
+        # The same kernel in SM cycles, so the power cap's clock is visible:
+        # its time x the median SM clock of the timed region, against the
+        # tensor pipe's own floor (dense bf16: 8192 flops per SM per clock on
+        # every SM; the E4M3 path issues twice the flops at twice the rate)
+        sms = torch.cuda.get_device_properties(local).multi_processor_count
+        mhz = (clocks or {}).get("sm_mhz")
+        if mhz:
+            kc = head_ms * 1e3 * mhz / 1e3
+            mma_kc = flops / (sms * 8192.0) / 1e3
+            roof["cycles"] = {"kernel_kcycles": kc, "mma_floor_kcycles": mma_kc, "mma_frac_of_cycles": mma_kc / kc,
+                              "clock_mhz": mhz, "what": "kernel_us x median SM clock of the timed region; "
+                              "floor = 2 R d V flops / (SMs x 8192 dense bf16 flops per clock)"}
         if B == 1:
             k_desc = "k cycling 0/23/47"
         else:
