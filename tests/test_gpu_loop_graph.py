@@ -266,5 +266,10 @@ def test_loop_graph_handle_runs_again_and_equals_the_one_shot_loop():
                              has_prev=hp0.copy())
             _same(got, ref)
             assert int(state.k.item()) == int(steps.max()) + k_start
+        # a first step outside the schedule is refused before any launch
+        with pytest.raises(dg.DGError) as ei:
+            lg.run(np.zeros(B, np.uint8), k_start=params.max_steps)
+        assert ei.value.code == 4                       # DG_ERR_RANGE
     finally:
         lg.close()
+    lg.close()                                          # closing twice is harmless
