@@ -163,12 +163,15 @@ class ClockSampler:
                 return None
         sm = [num(r[1]) for r in rows if num(r[1]) is not None]
         mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        # board power of the samples taken under load (SM clock above idle)
+        pw = [num(r[3]) for r in rows if num(r[3]) is not None and num(r[1]) is not None and num(r[1]) > 600]
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
         reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip().lower() == "active"})
         # samples while the GPU was busy (clock above idle) describe the load
         busy = [s for s in sm if s > 600] or sm
         return {"sm_mhz": statistics.median(busy) if busy else None,
                 "sm_max_mhz": max(mx) if mx else None,
+                "power_w": statistics.median(pw) if pw else None,
                 "reasons": reasons, "samples": len(sm)}
 
 

@@ -27,7 +27,7 @@ def test_summary_takes_the_busy_median_and_collects_reasons():
             _row("2026/12/03 01:00:00.150", 1300, 1965)]
     s = bench.ClockSampler.summarize(rows)
     assert s["sm_mhz"] == 1200 and s["sm_max_mhz"] == 1965 and s["samples"] == 4
-    assert s["reasons"] == ["sw_power_cap"]
+    assert s["reasons"] == ["sw_power_cap"] and s["power_w"] == 500.0
 
 
 def test_window_selects_rows_by_timestamp():
