@@ -680,6 +680,12 @@ def main():
             "us_per_step": ms_per_step * 1e3,
             "roofline": roof,
             "clocks": clocks,
+            # the board runs at its power limit: energy per step = median
+            # board power under load x step time
+            "energy": ({"mj_per_step": clocks["power_w"] * ms_per_step, "power_w": clocks["power_w"],
+                        "how": "per GPU (rank 0's): median nvidia-smi power.draw of the timed region's samples "
+                               "under load x ms_per_step"}
+                       if clocks and clocks.get("power_w") else None),
             "e2e": {"value": e2e_value, "unit": "slots/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                     "how": "h uploaded from pinned host memory every step (the next step's upload overlapping "
