@@ -220,9 +220,9 @@ dg_status dg_denoise_loop(const dg_shape* shape, const dg_params* params,
                           int32_t* argmax, int32_t* stop,
                           void* workspace, size_t ws_bytes, void* stream);
 
-/* ---- self-conditioning signal ([Report] Table 1: a 7.8M-parameter MLP
- * "for self-conditioning"; the pages define neither the signal nor the
- * MLP).  Reading: the signal of slot r is the embedding expected under the
+/* ---- self-conditioning signal ([Report] Table 1: the model carries a
+ * 7.8M-parameter self-conditioning MLP; the pages define neither the signal
+ * nor the MLP).  Reading: the signal of slot r is the embedding expected under the
  * step's tempered distribution, s[r] = sum_v softmax(z[r] / tau_k)_v E[v]
  * (a d-vector per slot), the input such an MLP would project.  The MLP has
  * trained weights and is out of scope.
